@@ -1,0 +1,142 @@
+/*
+ * tpmlp — tensor-parallel Transformer MLP block on one B200 (sm_100a).
+ *
+ * The block is Z = GeLU(X·A + a)·B + b with A (h × F) split by columns into p
+ * shards and B (F × h) split by rows into the matching p shards, forward and
+ * backward (page "Megatron", zzmblog.top, section "张量并行 / 数学原理" for the
+ * two splits; section "Transformer层的张量并行实现" for their pairing in the MLP;
+ * section "实战使用 / 基础训练示例" for activation_func = "gelu"). All p shards
+ * live on one GPU, so the all-reduce of the row-parallel partials happens
+ * inside the library as an ordered shard reduction.
+ *
+ * Conventions for every entry point below:
+ *  - Matrices are dense, row-major, with no padding between rows.
+ *  - Pointers are DEVICE pointers owned by the caller, except where a
+ *    comment says otherwise. The library never allocates or frees memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *    stream). Work is enqueued asynchronously on it; the call returns once
+ *    the launches are enqueued.
+ *  - All argument checks happen before the first launch: a call that
+ *    returns an error has enqueued nothing.
+ *  - Results are deterministic: the same inputs and p give bit-identical
+ *    outputs on every run.
+ *  - The library keeps a small amount of process-wide state (the split
+ *    policy, the wait limit, a launch counter, one device status word per
+ *    device); calls from several host threads at once are not supported.
+ */
+#ifndef TPMLP_H
+#define TPMLP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum tpmlp_status {
+    TPMLP_OK = 0,
+    TPMLP_ERR_INVALID = 1,     /* bad size, p, null pointer or dtype code */
+    TPMLP_ERR_ALIGN = 2,       /* a bf16 pointer is not 16-byte aligned */
+    TPMLP_ERR_UNSUPPORTED = 3, /* no GPU of compute capability 10.x, or sizes beyond int32 */
+    TPMLP_ERR_WORKSPACE = 4,   /* workspace null or smaller than tpmlp_workspace_size() */
+    TPMLP_ERR_CUDA = 5,        /* a CUDA runtime/driver call or a launch failed */
+    TPMLP_ERR_TIMEOUT = 6      /* a kernel gave up a bounded wait (device status word) */
+} tpmlp_status;
+
+/* Element type of X, A, a, B, b, H, Y, Z, dZ, dH and dX. Weight and bias
+ * gradients (dA, da, dB, db) are always fp32 ("weight update in full
+ * precision", page "Megatron", section "其他关键技术 / 混合精度训练").
+ * TPMLP_BF16 accumulates in fp32 on the tensor cores; TPMLP_FP32 uses fp32
+ * FFMA throughout (no TF32). */
+typedef enum tpmlp_dtype { TPMLP_BF16 = 0, TPMLP_FP32 = 1 } tpmlp_dtype;
+
+/* Bytes of device workspace that tp_mlp_fwd and tp_mlp_bwd need for these
+ * sizes under the current split policy (the larger of the two calls' needs).
+ * Returns 0 for invalid sizes. Holds the fp32 shard partials of the two
+ * row-parallel products when they are split by shard, and the partial column
+ * sums of the bias gradients. */
+size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt);
+
+/* Forward (column-parallel, then row-parallel):
+ *   H[:, i·Fp:(i+1)·Fp] = X·A_i + a_i        for shard i = 1..p, Fp = F/p
+ *   Y = GeLU(H) = ½·H·(1 + erf(H/√2))         (exact erf form)
+ *   Z = Σ_{i=1..p} Y_i·B_i + b                summed over shards in ascending i
+ * X: T×h. A: h×F. a: F (may be NULL = zero). B: F×h. b: h (may be NULL).
+ * H, Y: T×F outputs (H, the pre-activation, and Y are both kept for the
+ * backward). Z: T×h output. All of dtype `dt`.
+ * Requires T ≥ 0, h ≥ 1, F ≥ 1, p ≥ 1, F % p == 0. For TPMLP_BF16 the
+ * pointers must be 16-byte aligned; when h % 8 != 0 or F % 8 != 0 a plain
+ * (slower) GPU kernel path serves the call.
+ * workspace: device buffer of at least tpmlp_workspace_size() bytes (may be
+ * NULL when that size is 0). */
+tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void* B,
+                        const void* b, void* H, void* Y, void* Z, int64_t T, int64_t h,
+                        int64_t F, int p, tpmlp_dtype dt, void* workspace,
+                        size_t workspace_bytes, void* stream);
+
+/* Backward, given the upstream gradient dZ (T×h) and the forward's X, A, B,
+ * H and Y (chain rule on the forward above):
+ *   db = 1ᵀ·dZ                       (h, fp32)
+ *   dB_i = Y_iᵀ·dZ                   (F×h, fp32; row block i per shard)
+ *   dH_i = (dZ·B_iᵀ) ⊙ GeLU′(H_i)    (T×F, dtype dt; written to dH)
+ *   da = 1ᵀ·dH                       (F, fp32)
+ *   dA_i = Xᵀ·dH_i                   (h×F, fp32; column block i per shard)
+ *   dX = Σ_{i=1..p} dH_i·A_iᵀ        (T×h, dtype dt; ascending i)
+ * GeLU′(x) = Φ(x) + x·φ(x). X is replicated across shards, so its gradient
+ * is the sum over shards: the backward counterpart of the forward all-reduce.
+ * dH is an output the caller owns (T×F). Same requirements as tp_mlp_fwd.
+ * With T == 0 the gradients dA, da, dB, db are set to zero. */
+tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void* B,
+                        const void* H, const void* Y, void* dX, float* dA, float* da,
+                        float* dB, float* db, void* dH, int64_t T, int64_t h, int64_t F,
+                        int p, tpmlp_dtype dt, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+/* Static, NUL-terminated description of a status code. */
+const char* tpmlp_strerror(tpmlp_status s);
+
+/* Synchronizes `stream`, then reads and clears the current device's status
+ * word. Returns TPMLP_ERR_TIMEOUT if a kernel launched since the last read
+ * gave up a bounded wait (its outputs are then undefined), TPMLP_ERR_CUDA if
+ * the synchronization itself failed, else TPMLP_OK. */
+tpmlp_status tpmlp_last_device_status(void* stream);
+
+/* How the two row-parallel products (Z = Σ Y_i·B_i and dX = Σ dH_i·A_iᵀ)
+ * are scheduled on the tensor-core path:
+ *   0 = automatic (split by shard only when the output tiles alone cannot
+ *       fill the GPU),
+ *   1 = never split: each output tile loops over all shards in ascending
+ *       order, accumulating in tensor memory,
+ *   2 = always split by shard when F/p is a multiple of 64: each shard's
+ *       partial is written in fp32 and the partials are summed in ascending
+ *       shard order, then the bias is added.
+ * Both orders are deterministic; results agree within rounding. Returns
+ * TPMLP_ERR_INVALID for other values. The workspace size depends on it. */
+tpmlp_status tpmlp_set_split_policy(int policy);
+int tpmlp_get_split_policy(void);
+
+/* Upper bound, in nanoseconds, on any single wait inside a kernel (for data
+ * from the tensor-memory accelerator, for the tensor cores, between warps).
+ * Default 2e9 (2 s). A wait that runs out sets the device status word to
+ * TPMLP_ERR_TIMEOUT and the kernel winds down and returns. 0 restores the
+ * default. */
+void tpmlp_set_wait_limit_ns(uint64_t ns);
+
+/* Launches one kernel that waits, with limit `limit_ns`, on a barrier that
+ * nothing ever completes, so that the bounded-wait path can be tested: after
+ * it, tpmlp_last_device_status() returns TPMLP_ERR_TIMEOUT and the context
+ * stays usable. */
+tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t tpmlp_launch_count(void);
+
+/* Library version, major·10000 + minor·100 + patch. */
+int tpmlp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TPMLP_H */

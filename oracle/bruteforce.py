@@ -1,0 +1,47 @@
+"""Pure-Python brute-force evaluation of the MLP block, for tiny shapes only.
+
+TEST INFRASTRUCTURE ONLY. It shares nothing with the C oracle: each entry is
+an explicit dot product summed with ``math.fsum`` (correctly rounded sum) and
+GeLU uses ``math.erf``. It exists to pin the C oracle on shapes up to about
+T = 8, h = 6, F = 24.
+
+Definitions (page "Megatron", zzmblog.top, section "张量并行 / 数学原理";
+activation "gelu" from the training script's TransformerConfig):
+H = X·A + a, Y = GeLU(H), Z = Y·B + b; the gradients follow the chain rule.
+"""
+from __future__ import annotations
+
+import math
+
+
+def _phi_cdf(x: float) -> float:
+    return 0.5 * (1.0 + math.erf(x / math.sqrt(2.0)))
+
+
+def _gelu(x: float) -> float:
+    return x * _phi_cdf(x)
+
+
+def _gelu_grad(x: float) -> float:
+    return _phi_cdf(x) + x * math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
+
+
+def mlp(X, A, a, B, b, dZ):
+    """X: T×h, A: h×F, a: F, B: F×h, b: h, dZ: T×h, as nested lists of floats.
+
+    Returns a dict of nested lists: H, Y, Z, dH, dX, dA, da, dB, db.
+    """
+    T, h, F = len(X), len(X[0]), len(A[0])
+    H = [[math.fsum([X[t][k] * A[k][f] for k in range(h)] + [a[f]]) for f in range(F)]
+         for t in range(T)]
+    Y = [[_gelu(H[t][f]) for f in range(F)] for t in range(T)]
+    Z = [[math.fsum([Y[t][f] * B[f][j] for f in range(F)] + [b[j]]) for j in range(h)]
+         for t in range(T)]
+    db = [math.fsum(dZ[t][j] for t in range(T)) for j in range(h)]
+    dB = [[math.fsum(Y[t][f] * dZ[t][j] for t in range(T)) for j in range(h)] for f in range(F)]
+    dY = [[math.fsum(dZ[t][j] * B[f][j] for j in range(h)) for f in range(F)] for t in range(T)]
+    dH = [[dY[t][f] * _gelu_grad(H[t][f]) for f in range(F)] for t in range(T)]
+    da = [math.fsum(dH[t][f] for t in range(T)) for f in range(F)]
+    dA = [[math.fsum(X[t][k] * dH[t][f] for t in range(T)) for f in range(F)] for k in range(h)]
+    dX = [[math.fsum(dH[t][f] * A[k][f] for f in range(F)) for k in range(h)] for t in range(T)]
+    return dict(H=H, Y=Y, Z=Z, dH=dH, dX=dX, dA=dA, da=da, dB=dB, db=db)
