@@ -1,0 +1,443 @@
+#!/usr/bin/env python
+"""Bench of the tensor-parallel MLP block: forward + backward TFLOP/s on B200.
+
+One step = tp_mlp_fwd + tp_mlp_bwd over one batch of seeded synthetic input
+(the whole hot path: column GEMM with bias+GeLU, row GEMM with the ordered
+shard sum, bias-gradient column sums, dgrad with GeLU′, two weight-gradient
+GEMMs, dgrad of X with the ordered shard sum). FLOPs counted = 12·T·h·F per
+step (the six T·h·F products); elementwise and reduction work is in the time
+but not in the count.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 7b]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, bounded sample
+
+With N > 1 (launched by torch.distributed.run) every rank runs an
+independent replica of the workload (the block is not sharded across GPUs):
+weak scaling, value = all ranks' FLOPs / the slowest rank's time.
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import hashlib
+import io
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TP-MLP fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+UNIT = "TFLOP/s"
+DATASHEET_BF16_DENSE_TFLOPS = 2250.0  # NVIDIA B200 datasheet (HGX B200), dense BF16
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="7b")
+    ap.add_argument("--e2e-steps", type=int, default=20)
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle CPU baseline (for profiler runs)")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0,
+                    help="target seconds of oracle work for the CPU baseline sample")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    return args
+
+
+# ----------------------------------------------------------- distributed glue
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+
+
+def max_over_ranks(x: float, device=None) -> float:
+    """Largest value of x over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def sum_over_ranks(x: float, device=None) -> float:
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier():
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.barrier()
+
+
+def aggregate(flops_per_step_per_rank: float, steps: int, max_seconds: float, world: int) -> dict:
+    """Whole-job throughput of `world` replicas that each ran `steps` steps,
+    timed by the slowest rank."""
+    total = flops_per_step_per_rank * steps * world
+    return {"value": total / max_seconds / 1e12, "ms_per_step": 1e3 * max_seconds / steps}
+
+
+# ------------------------------------------------------------------- peaks
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "tensor_transformer_mlp_block_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_for(kind: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources for this workload; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+        e = t[workload][kind]
+        if e.get("source_hash") != source_hash():
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ------------------------------------------------------------------ clocks
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons in the background."""
+
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(self.gpu_index), "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self, t0: float, t1: float) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for r in csv.reader(f):
+                if len(r) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    rows.append((ts, [c.strip() for c in r]))
+                except Exception:
+                    continue
+        os.unlink(self.path)
+        inside = [c for ts, c in rows if t0 - 1.0 <= ts <= t1 + 1.0] or [c for _, c in rows]
+        if not inside:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(c[2]) for c in inside if c[2].replace(".", "").isdigit()]
+        smax = [float(c[3]) for c in inside if c[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for c in inside for i in range(4) if c[6 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(inside),
+                "power_w_max": max((float(c[4]) for c in inside if c[4].replace(".", "").isdigit()),
+                                   default=None)}
+
+
+def physical_gpu_index(local_rank: int) -> int:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        parts = [p.strip() for p in vis.split(",") if p.strip()]
+        if local_rank < len(parts) and parts[local_rank].isdigit():
+            return int(parts[local_rank])
+    return local_rank
+
+
+# ------------------------------------------------------------ CPU baseline
+
+def cpu_baseline(inp: dict, cfg, target_seconds: float) -> dict:
+    """The fp64 oracle, as it stands, on a bounded sample of the workload:
+    token rows R (forward and dX for those rows) and hidden columns J (H, dH,
+    dA, dB for those columns). Rate = the sample's algorithmic flops / wall
+    time on this host's cores."""
+    import numpy as np
+
+    import oracle
+    from tensor_transformer_mlp_block_b200.inputs import sample_indices
+    n = {k: v.to(dtype=__import__("torch").float64).numpy() for k, v in inp.items()}
+
+    def run(n_r, n_j):
+        R = sample_indices(cfg.T, n_r, seed=1234).numpy()[:n_r]
+        J = sample_indices(cfg.F, n_j, seed=1235).numpy()[:n_j]
+        t0 = time.perf_counter()
+        oracle.rows(n["X"], n["A"], n["a"], n["B"], n["b"], n["dZ"], R)
+        oracle.cols(n["X"], n["A"][:, J], n["a"][J], n["B"][J, :], n["dZ"], np.arange(len(J)))
+        dt = time.perf_counter() - t0
+        flops = 8.0 * cfg.h * cfg.F * len(R) + 8.0 * cfg.T * cfg.h * len(J)
+        return dt, flops, len(R), len(J)
+
+    dt, fl, _, _ = run(2, 2)
+    rate = fl / max(dt, 1e-9)
+    per_unit = 8.0 * cfg.h * cfg.F + 8.0 * cfg.T * cfg.h
+    k = max(2, int(target_seconds * rate / per_unit))
+    k = min(k, cfg.T, cfg.F)
+    dt, fl, nr, nj = run(k, k)
+    return {"value": fl / dt / 1e12, "unit": UNIT, "cores": oracle.get_threads(), "kind": "oracle",
+            "sample": f"{nr} token rows + {nj} hidden columns of the {cfg.name} workload "
+                      f"({fl / 1e9:.1f} GFLOP fp64 in {dt:.1f} s)",
+            "seconds": dt}
+
+
+# --------------------------------------------------------------- our arm
+
+def bench_ours(args, cfg, world, rank, local):
+    import torch
+
+    from tensor_transformer_mlp_block_b200 import binding
+    from tensor_transformer_mlp_block_b200.inputs import make_inputs, torch_dtype
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist_init(world, "nccl")
+    peaks, peaks_src = load_peaks()
+
+    inp = make_inputs(cfg)
+    d = {k: v.to(dev) for k, v in inp.items()}
+    dt = torch_dtype(cfg.dtype)
+    T, h, F, p = cfg.T, cfg.h, cfg.F, cfg.p
+    f32 = torch.float32
+    H = torch.empty((T, F), dtype=dt, device=dev)
+    Y = torch.empty((T, F), dtype=dt, device=dev)
+    Z = torch.empty((T, h), dtype=dt, device=dev)
+    gout = dict(dX=torch.empty((T, h), dtype=dt, device=dev), dA=torch.empty((h, F), dtype=f32, device=dev),
+                da=torch.empty((F,), dtype=f32, device=dev), dB=torch.empty((F, h), dtype=f32, device=dev),
+                db=torch.empty((h,), dtype=f32, device=dev), dH=torch.empty((T, F), dtype=dt, device=dev))
+    ws = torch.empty(max(binding.workspace_size(T, h, F, p, dt), 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(x=None, dz=None):
+        x = d["X"] if x is None else x
+        dz = d["dZ"] if dz is None else dz
+        binding.forward(x, d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, Z), workspace=ws)
+        binding.backward(dz, x, d["A"], d["B"], H, Y, p, out=gout, workspace=ws)
+
+    working_set = sum(t.numel() * t.element_size() for t in [*d.values(), H, Y, Z, *gout.values()])
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+
+    sampler = ClockSampler(physical_gpu_index(local))
+    sampler.start()
+    time.sleep(1.0)
+    binding.profile_reset()
+    binding.profile_enable(True)
+    launches0 = binding.launch_count()
+    barrier()
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    barrier()
+    t_wall1 = time.time()
+    launches = binding.launch_count() - launches0
+    binding.profile_enable(False)
+    kinds = binding.profile_collect()
+    clocks = sampler.stop(t_wall0, t_wall1)
+    status = binding.last_device_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    seconds = e0.elapsed_time(e1) / 1e3
+    max_seconds = max_over_ranks(seconds, dev)
+    agg = aggregate(cfg.flops_fwd_bwd, args.steps, max_seconds, world)
+
+    # dominant kernel and its roofline (tensor-bound: algorithmic flops / event time)
+    top_name, top = max(kinds.items(), key=lambda kv: kv[1]["ms"])
+    per_launch_ms = top["ms"] / top["launches"]
+    achieved = top["flops"] / top["launches"] / (per_launch_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops_sustained"]
+    roofline = {"bound": "tensor", "kernel": top_name, "achieved": achieved, "peak": peak,
+                "unit": "TFLOP/s", "frac": achieved / peak,
+                "traffic": traffic_for(top_name, cfg.name),
+                "peak_source": f"{peaks_src} bf16 sustained (kernel timed inside a long step loop)",
+                "launches": top["launches"], "ms_per_launch": per_launch_ms,
+                "share_of_step": top["ms"] / sum(k["ms"] for k in kinds.values())}
+    per_kernel = {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / v["launches"],
+                      "tflops": (v["flops"] / v["ms"] / 1e9) if v["flops"] else None,
+                      "gbs": v["bytes"] / v["ms"] / 1e6}
+                  for k, v in kinds.items()}
+
+    # end to end through the public API with pinned host buffers
+    hX = inp["X"].pin_memory()
+    hdZ = inp["dZ"].pin_memory()
+    hZ = torch.empty((T, h), dtype=dt).pin_memory()
+    hdX = torch.empty((T, h), dtype=dt).pin_memory()
+    xin = torch.empty_like(d["X"])
+    dzin = torch.empty_like(d["dZ"])
+
+    def e2e_step():
+        xin.copy_(hX, non_blocking=True)
+        dzin.copy_(hdZ, non_blocking=True)
+        step(xin, dzin)
+        hZ.copy_(Z, non_blocking=True)
+        hdX.copy_(gout["dX"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_max = max_over_ranks(e0.elapsed_time(e1) / 1e3, dev)
+    e2e_val = aggregate(cfg.flops_fwd_bwd, args.e2e_steps, e2e_max, world)["value"]
+    bytes_in = hX.numel() * hX.element_size() + hdZ.numel() * hdZ.element_size()
+    bytes_out = hZ.numel() * hZ.element_size() + hdX.numel() * hdX.element_size()
+
+    line = {
+        "metric": METRIC, "value": agg["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "fp32",
+        "data": "synthetic (seeded Gaussian inputs, random-init weights of the named shapes)",
+        "config": {"workload": f"{cfg.name}-class TP-MLP fwd+bwd", "T": T, "h": h, "F": F, "p": p,
+                   "flops_per_step": cfg.flops_fwd_bwd, "parallelism": f"replicas x{world}",
+                   "l2": f"working set {working_set / 2**30:.2f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB "
+                         "(inputs larger than L2; no flush)"},
+        "frac_of_peak": {"measured_burst": agg["value"] / world / peaks["bf16_tflops"],
+                         "measured_sustained": agg["value"] / world / peaks["bf16_tflops_sustained"],
+                         "datasheet_dense": agg["value"] / world / DATASHEET_BF16_DENSE_TFLOPS,
+                         "peaks": peaks_src},
+        "roofline": roofline,
+        "kernels": per_kernel,
+        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": bytes_in,
+                "d2h_bytes_per_step": bytes_out, "steps": args.e2e_steps,
+                "what": "per step: X and dZ copied in from pinned host memory, fwd+bwd, Z and dX "
+                        "copied out; weights and weight gradients stay resident"},
+        "gpu_launches": launches,
+        "clocks": clocks,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inp, cfg, args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    return line
+
+
+# ---------------------------------------------------------- reference arm
+
+def bench_reference(args, cfg, world, rank):
+    """The fp64 oracle on the host cores: each step is a bounded sample of the
+    workload (token rows + hidden columns), so K + W steps end in minutes."""
+    if rank != 0:
+        return None
+    from tensor_transformer_mlp_block_b200.inputs import make_inputs
+    inp = make_inputs(cfg)
+    per_step = max(0.2, min(10.0, 120.0 / (args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_baseline(inp, cfg, per_step)
+    total_flops, total_s, last = 0.0, 0.0, None
+    for _ in range(args.steps):
+        last = cpu_baseline(inp, cfg, per_step)
+        total_s += last["seconds"]
+        total_flops += last["value"] * 1e12 * last["seconds"]
+    value = total_flops / total_s / 1e12
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded Gaussian inputs)",
+        "config": {"workload": f"{cfg.name}-class TP-MLP fwd+bwd", "T": cfg.T, "h": cfg.h,
+                   "F": cfg.F, "p": cfg.p},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": last["cores"], "kind": "oracle",
+                         "sample": "per step: " + last["sample"]},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    from tensor_transformer_mlp_block_b200 import configs
+    cfg = configs.get(args.config)
+    world, rank, local = dist_env()
+    if args.gpus != world and world > 1:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE {world}", file=sys.stderr)
+    if args.impl == "reference":
+        line = bench_reference(args, cfg, world, rank)
+    else:
+        line = bench_ours(args, cfg, world, rank, local)
+    if rank == 0 and line is not None:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized():
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -132,6 +132,25 @@ tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream);
 /* Number of kernels this library has launched in this process. */
 uint64_t tpmlp_launch_count(void);
 
+/* Per-kernel timing on the launching stream, for measurement tools. While
+ * enabled (on != 0), every kernel launch is bracketed by a pair of CUDA
+ * events on its stream and tagged with its step (F1 column GEMM, F2 row
+ * GEMM, B1..B5, and the helper kernels). tpmlp_profile_collect() waits for
+ * the recorded events and adds their elapsed times into per-kind totals,
+ * together with each launch's algorithmic flops (2·M·N·K for a GEMM) and
+ * algorithmic bytes (every operand read once, every output written once).
+ * Returns the number of kinds, or -1 if a CUDA call failed.
+ * tpmlp_profile_read(kind, ...) returns those totals (any out-pointer may be
+ * NULL); tpmlp_profile_name(kind) its static name; tpmlp_profile_reset()
+ * clears them. Not thread-safe. */
+void tpmlp_profile_enable(int on);
+int tpmlp_profile_collect(void);
+int tpmlp_profile_kinds(void);
+const char* tpmlp_profile_name(int kind);
+tpmlp_status tpmlp_profile_read(int kind, uint64_t* launches, double* total_ms, double* flops,
+                                double* bytes);
+void tpmlp_profile_reset(void);
+
 /* Library version, major·10000 + minor·100 + patch. */
 int tpmlp_version(void);
 

@@ -1,0 +1,255 @@
+"""Python binding of ``libtpmlp.so`` (ctypes). Argument marshalling only.
+
+Every step of the block runs in the library's CUDA kernels; torch supplies
+device memory (the output and workspace tensors) and the current stream.
+There is no other implementation behind these functions: if the library is
+missing or the tensors are not on a CUDA device, they raise.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+
+import torch
+
+from .build import LIB as _LIB_PATH
+
+OK, ERR_INVALID, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
+BF16, FP32 = 0, 1
+
+# The entry points include/tpmlp.h declares, in declaration order.
+EXPORTS = (
+    "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tpmlp_strerror",
+    "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
+    "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count",
+    "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
+    "tpmlp_profile_read", "tpmlp_profile_reset", "tpmlp_version",
+)
+
+_lib = None
+_lock = threading.Lock()
+
+
+class TPMLPError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {strerror(status)} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libtpmlp.so (once). Raises if it has not been built."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(_LIB_PATH):
+                raise RuntimeError(
+                    f"CUDA library {_LIB_PATH} is missing; build it with "
+                    "`python -m tensor_transformer_mlp_block_b200.build`")
+            L = ctypes.CDLL(_LIB_PATH)
+            vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
+            L.tpmlp_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
+            L.tpmlp_workspace_size.restype = sz
+            L.tp_mlp_fwd.argtypes = [vp] * 8 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
+            L.tp_mlp_fwd.restype = ctypes.c_int
+            L.tp_mlp_bwd.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
+            L.tp_mlp_bwd.restype = ctypes.c_int
+            L.tpmlp_strerror.argtypes = [ctypes.c_int]
+            L.tpmlp_strerror.restype = ctypes.c_char_p
+            L.tpmlp_last_device_status.argtypes = [vp]
+            L.tpmlp_last_device_status.restype = ctypes.c_int
+            L.tpmlp_set_split_policy.argtypes = [ctypes.c_int]
+            L.tpmlp_set_split_policy.restype = ctypes.c_int
+            L.tpmlp_get_split_policy.restype = ctypes.c_int
+            L.tpmlp_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
+            L.tpmlp_set_wait_limit_ns.restype = None
+            L.tpmlp_wait_selftest.argtypes = [ctypes.c_uint64, vp]
+            L.tpmlp_wait_selftest.restype = ctypes.c_int
+            L.tpmlp_launch_count.restype = ctypes.c_uint64
+            L.tpmlp_version.restype = ctypes.c_int
+            L.tpmlp_profile_enable.argtypes = [ctypes.c_int]
+            L.tpmlp_profile_enable.restype = None
+            L.tpmlp_profile_collect.restype = ctypes.c_int
+            L.tpmlp_profile_kinds.restype = ctypes.c_int
+            L.tpmlp_profile_name.argtypes = [ctypes.c_int]
+            L.tpmlp_profile_name.restype = ctypes.c_char_p
+            L.tpmlp_profile_read.argtypes = [ctypes.c_int, ctypes.POINTER(ctypes.c_uint64)] + \
+                [ctypes.POINTER(ctypes.c_double)] * 3
+            L.tpmlp_profile_read.restype = ctypes.c_int
+            L.tpmlp_profile_reset.restype = None
+            _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().tpmlp_strerror(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise TPMLPError(status, where)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return FP32
+    raise TypeError(f"unsupported dtype {t.dtype}; use bfloat16 or float32")
+
+
+def _stream_ptr(device: torch.device, stream) -> int:
+    s = torch.cuda.current_stream(device) if stream is None else stream
+    return s.cuda_stream
+
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype, device) -> None:
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def workspace_size(T: int, h: int, F: int, p: int, dtype: torch.dtype = torch.bfloat16) -> int:
+    code = BF16 if dtype == torch.bfloat16 else FP32
+    return int(lib().tpmlp_workspace_size(T, h, F, p, code))
+
+
+def _workspace(T, h, F, p, dtype, device, workspace):
+    n = workspace_size(T, h, F, p, dtype)
+    if workspace is None:
+        return torch.empty(max(n, 1), dtype=torch.uint8, device=device), n
+    if workspace.numel() * workspace.element_size() < n:
+        raise ValueError(f"workspace has {workspace.nbytes} bytes, needs {n}")
+    return workspace, workspace.numel() * workspace.element_size()
+
+
+def forward(X, A, a, B, b, p: int, *, out=None, workspace=None, stream=None):
+    """H, Y, Z of Z = GeLU(X·A + a)·B + b with A, B split into p shards.
+
+    X: T×h, A: h×F, a: F or None, B: F×h, b: h or None, all bf16 (or all
+    fp32) CUDA tensors. Returns (H, Y, Z); `out` may supply them."""
+    T, h = X.shape
+    F = A.shape[1]
+    dt, dev = X.dtype, X.device
+    _need(X, "X", (T, h), dt, dev)
+    _need(A, "A", (h, F), dt, dev)
+    _need(B, "B", (F, h), dt, dev)
+    if a is not None:
+        _need(a, "a", (F,), dt, dev)
+    if b is not None:
+        _need(b, "b", (h,), dt, dev)
+    if out is None:
+        H = torch.empty((T, F), dtype=dt, device=dev)
+        Y = torch.empty((T, F), dtype=dt, device=dev)
+        Z = torch.empty((T, h), dtype=dt, device=dev)
+    else:
+        H, Y, Z = out
+        _need(H, "H", (T, F), dt, dev)
+        _need(Y, "Y", (T, F), dt, dev)
+        _need(Z, "Z", (T, h), dt, dev)
+    ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
+    st = lib().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(a), _ptr(B), _ptr(b), _ptr(H), _ptr(Y), _ptr(Z),
+                          T, h, F, int(p), _dtype_code(X), _ptr(ws), ws_bytes,
+                          _stream_ptr(dev, stream))
+    _check(st, "tp_mlp_fwd")
+    return H, Y, Z
+
+
+def backward(dZ, X, A, B, H, Y, p: int, *, out=None, workspace=None, stream=None):
+    """Gradients of the block for upstream gradient dZ (T×h).
+
+    Returns a dict: dX (T×h, input dtype), dA (h×F, fp32), da (F, fp32),
+    dB (F×h, fp32), db (h, fp32), dH (T×F, input dtype)."""
+    T, h = X.shape
+    F = A.shape[1]
+    dt, dev = X.dtype, X.device
+    for name, t, shp in (("dZ", dZ, (T, h)), ("X", X, (T, h)), ("A", A, (h, F)), ("B", B, (F, h)),
+                         ("H", H, (T, F)), ("Y", Y, (T, F))):
+        _need(t, name, shp, dt, dev)
+    f32 = torch.float32
+    if out is None:
+        out = dict(dX=torch.empty((T, h), dtype=dt, device=dev),
+                   dA=torch.empty((h, F), dtype=f32, device=dev),
+                   da=torch.empty((F,), dtype=f32, device=dev),
+                   dB=torch.empty((F, h), dtype=f32, device=dev),
+                   db=torch.empty((h,), dtype=f32, device=dev),
+                   dH=torch.empty((T, F), dtype=dt, device=dev))
+    for name, shp, d in (("dX", (T, h), dt), ("dA", (h, F), f32), ("da", (F,), f32),
+                         ("dB", (F, h), f32), ("db", (h,), f32), ("dH", (T, F), dt)):
+        _need(out[name], name, shp, d, dev)
+    ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
+    st = lib().tp_mlp_bwd(_ptr(dZ), _ptr(X), _ptr(A), _ptr(B), _ptr(H), _ptr(Y), _ptr(out["dX"]),
+                          _ptr(out["dA"]), _ptr(out["da"]), _ptr(out["dB"]), _ptr(out["db"]),
+                          _ptr(out["dH"]), T, h, F, int(p), _dtype_code(X), _ptr(ws), ws_bytes,
+                          _stream_ptr(dev, stream))
+    _check(st, "tp_mlp_bwd")
+    return out
+
+
+def set_split_policy(policy: int) -> None:
+    _check(lib().tpmlp_set_split_policy(int(policy)), "tpmlp_set_split_policy")
+
+
+def get_split_policy() -> int:
+    return int(lib().tpmlp_get_split_policy())
+
+
+def set_wait_limit_ns(ns: int) -> None:
+    lib().tpmlp_set_wait_limit_ns(int(ns))
+
+
+def last_device_status(stream=None, device=None) -> int:
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    return int(lib().tpmlp_last_device_status(_stream_ptr(dev, stream)))
+
+
+def wait_selftest(limit_ns: int, stream=None) -> None:
+    dev = torch.device("cuda", torch.cuda.current_device())
+    _check(lib().tpmlp_wait_selftest(int(limit_ns), _stream_ptr(dev, stream)), "tpmlp_wait_selftest")
+
+
+def launch_count() -> int:
+    return int(lib().tpmlp_launch_count())
+
+
+def version() -> int:
+    return int(lib().tpmlp_version())
+
+
+def profile_enable(on: bool = True) -> None:
+    """Bracket every library launch with CUDA events on its stream."""
+    lib().tpmlp_profile_enable(1 if on else 0)
+
+
+def profile_reset() -> None:
+    lib().tpmlp_profile_reset()
+
+
+def profile_collect() -> dict:
+    """Wait for the recorded events; return {kind: dict(launches, ms, flops,
+    bytes)} accumulated since the last reset (kinds with launches only)."""
+    L = lib()
+    n = L.tpmlp_profile_collect()
+    if n < 0:
+        raise TPMLPError(ERR_CUDA, "tpmlp_profile_collect")
+    out = {}
+    for k in range(L.tpmlp_profile_kinds()):
+        cnt = ctypes.c_uint64()
+        ms, fl, by = ctypes.c_double(), ctypes.c_double(), ctypes.c_double()
+        _check(L.tpmlp_profile_read(k, ctypes.byref(cnt), ctypes.byref(ms), ctypes.byref(fl),
+                                    ctypes.byref(by)), "tpmlp_profile_read")
+        if cnt.value:
+            out[L.tpmlp_profile_name(k).decode()] = dict(launches=int(cnt.value), ms=ms.value,
+                                                         flops=fl.value, bytes=by.value)
+    return out

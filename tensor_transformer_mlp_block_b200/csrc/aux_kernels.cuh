@@ -1,0 +1,144 @@
+// Bandwidth-bound helper kernels: the ordered sum of split partials (the
+// on-chip counterpart of the all-reduce after the row-parallel product) and
+// deterministic column sums (the bias gradients).
+#pragma once
+
+#include "gemm_tc.cuh"
+
+namespace tpmlp {
+
+// out[m, n] = round( Σ_{s=0..S-1} ws[s][m, n] + bias[n] ), the partials
+// added in ascending s, then the bias once. Each thread handles 8
+// consecutive columns (N % 8 == 0; all pointers 16-byte aligned).
+__global__ void __launch_bounds__(256) reduce_splits_bf16_kernel(
+    const float* __restrict__ ws, int splits, int64_t plane, const __nv_bfloat16* __restrict__ bias,
+    __nv_bfloat16* __restrict__ out, int64_t M, int64_t N) {
+    const int64_t groups = M * (N / 8);
+    for (int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gi < groups;
+         gi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const int64_t e = gi * 8;
+        float4 lo = __ldg(reinterpret_cast<const float4*>(ws + e));
+        float4 hi = __ldg(reinterpret_cast<const float4*>(ws + e + 4));
+        float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        for (int s = 1; s < splits; ++s) {
+            const float* p = ws + s * plane + e;
+            lo = __ldg(reinterpret_cast<const float4*>(p));
+            hi = __ldg(reinterpret_cast<const float4*>(p + 4));
+            v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
+            v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
+        }
+        if (bias != nullptr) {
+            const int64_t n = e % N;
+            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(bias + n);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                float2 t = __bfloat1622float2(b2[i]);
+                v[2 * i] += t.x;
+                v[2 * i + 1] += t.y;
+            }
+        }
+        uint4 o;
+        __nv_bfloat162 r0 = __floats2bfloat162_rn(v[0], v[1]);
+        __nv_bfloat162 r1 = __floats2bfloat162_rn(v[2], v[3]);
+        __nv_bfloat162 r2 = __floats2bfloat162_rn(v[4], v[5]);
+        __nv_bfloat162 r3 = __floats2bfloat162_rn(v[6], v[7]);
+        o.x = *reinterpret_cast<uint32_t*>(&r0);
+        o.y = *reinterpret_cast<uint32_t*>(&r1);
+        o.z = *reinterpret_cast<uint32_t*>(&r2);
+        o.w = *reinterpret_cast<uint32_t*>(&r3);
+        *reinterpret_cast<uint4*>(out + e) = o;
+    }
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+// Column sums, pass 1. Block (32, 8): lane x covers columns
+// [blockIdx.x·256 + 8x, +8), row phase y walks rows chunk_begin + y, +8, ...
+// of chunk blockIdx.y; the 8 phases are then added in order y = 0..7 and
+// the chunk's sums written to partial[blockIdx.y][:]. Fixed assignment and
+// fixed order: the result is bit-reproducible.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ X, int64_t R,
+                                                            int64_t C, int64_t rows_per_chunk,
+                                                            float* __restrict__ partial) {
+    __shared__ float red[8][256];
+    const int64_t c0 = blockIdx.x * 256 + threadIdx.x * 8;
+    const int64_t r_begin = blockIdx.y * rows_per_chunk;
+    const int64_t r_end = min(R, r_begin + rows_per_chunk);
+    float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    if (VEC && c0 < C) {
+        // C % 8 == 0 and X 16-byte aligned: 8 columns are 16 (bf16) or 32 (fp32) bytes
+        for (int64_t r = r_begin + threadIdx.y; r < r_end; r += 8) {
+            const T* row = X + r * C + c0;
+            if constexpr (sizeof(T) == 2) {
+                float f[8];
+                unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(row)), f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] += f[i];
+            } else {
+                const float4 lo = __ldg(reinterpret_cast<const float4*>(row));
+                const float4 hi = __ldg(reinterpret_cast<const float4*>(row) + 1);
+                acc[0] += lo.x; acc[1] += lo.y; acc[2] += lo.z; acc[3] += lo.w;
+                acc[4] += hi.x; acc[5] += hi.y; acc[6] += hi.z; acc[7] += hi.w;
+            }
+        }
+    } else if (!VEC) {
+        for (int64_t r = r_begin + threadIdx.y; r < r_end; r += 8) {
+            const T* row = X + r * C;
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+                if (c0 + i < C) acc[i] += to_f32<T>(row[c0 + i]);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) red[threadIdx.y][threadIdx.x * 8 + i] = acc[i];
+    __syncthreads();
+    const int t = threadIdx.y * 32 + threadIdx.x;  // 0..255: one column each
+    const int64_t c = blockIdx.x * 256 + t;
+    if (c < C) {
+        float s = red[0][t];
+        for (int y = 1; y < 8; ++y) s += red[y][t];
+        partial[blockIdx.y * C + c] = s;
+    }
+}
+
+// Column sums, pass 2: out[c] = Σ_{chunk ascending} partial[chunk][c].
+__global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ partial,
+                                                          int chunks, int64_t C,
+                                                          float* __restrict__ out) {
+    const int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+    if (c >= C) return;
+    float s = 0.0f;
+    for (int k = 0; k < chunks; ++k) s += partial[k * C + c];
+    out[c] = s;
+}
+
+__global__ void zero_f32_kernel(float* __restrict__ p, int64_t n) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+        p[i] = 0.0f;
+}
+
+// A kernel that waits, bounded, on an mbarrier that nothing completes:
+// exercises the timeout path (status word set, clean return).
+__global__ void wait_selftest_kernel(uint64_t limit_ns) {
+    __shared__ __align__(8) uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(&bar), 1);
+        abort_flag = 0;
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        if (!mbar_wait_bounded(smem_u32(&bar), 0, &abort_flag, limit_ns)) raise_timeout(&abort_flag);
+    }
+    __syncthreads();
+}
+
+}  // namespace tpmlp

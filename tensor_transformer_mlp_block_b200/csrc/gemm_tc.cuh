@@ -1,0 +1,400 @@
+// Persistent tcgen05 GEMM for sm_100a with fused epilogues.
+//
+//   D[M, N] = Σ_k Aop[m, k] · Bop[k, n]      (bf16 operands, fp32 accumulate)
+//
+// Operands are row-major tensors in global memory read by TMA in either
+// orientation: Aop is "K-major" when stored as [M][K] and "MN-major" when
+// stored as [K][M] (the transposed operand of a weight-gradient product);
+// likewise Bop is K-major when stored as [N][K] and MN-major as [K][N]. The
+// tensor cores read both orientations directly from 128-byte-swizzled shared
+// memory, so no transposed copy is ever made.
+//
+// CTA organisation (192 threads, one CTA per SM, persistent over tiles):
+//   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) k-blocks
+//   warp 1      tensor-memory allocator and MMA issuer (one thread)
+//   warps 2..5  epilogue: tensor memory -> registers -> fused math -> global
+// The accumulator is double-buffered in tensor memory (2 × BN fp32 columns
+// of 128 lanes), so the epilogue of one tile overlaps the next tile's
+// main loop. Work units are (output tile, K split) pairs handed out
+// round-robin: unit u goes to CTA u mod gridDim.x.
+//
+// Every wait is bounded (mbar_wait_bounded); a wait that runs out records
+// a timeout in the device status word and the CTA winds down: the producer
+// waits for its copies in flight, the MMA thread for its tensor-core work,
+// and tensor memory is freed before the CTA exits.
+#pragma once
+
+#include "ptx.cuh"
+
+namespace tpmlp {
+
+enum EpiKind : int {
+    EPI_GELU = 0,       // out0 = H = acc + bias (bf16), out1 = Y = GeLU(H) (bf16)
+    EPI_BIAS = 1,       // out0 = acc + bias (element type); bias may be null
+    EPI_DGELU = 2,      // out0 = dH = acc · GeLU′(aux) (bf16), aux = saved H (bf16)
+    EPI_F32 = 3,        // out0 (fp32) + split · split_stride = acc
+};
+
+struct GemmArgs {
+    int M, N, K;
+    int num_m_blocks, num_n_blocks;
+    int splits;        // K splits; work units = tiles × splits
+    int kb_per_split;  // k-blocks of BK per split
+    int k_blocks;      // ceil(K / BK)
+    void* out0;
+    void* out1;
+    int64_t ld_out;        // row stride (elements) of out0, out1 and aux
+    int64_t split_stride;  // elements between per-split planes of out0 (EPI_F32)
+    const __nv_bfloat16* bias;
+    const __nv_bfloat16* aux;
+    uint64_t wait_limit_ns;
+};
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+constexpr int kGroupM = 16;  // m-blocks per raster group (L2 reuse of Bop)
+
+template <int BN>
+struct TileCfg {
+    static_assert(BN % 64 == 0 && BN >= 64 && BN <= 256, "BN must be 64..256, multiple of 64");
+    static constexpr int A_BYTES = kBM * kBK * 2;  // 16 KB
+    static constexpr int B_BYTES = BN * kBK * 2;
+    static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+    static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+    // tensor-memory columns: two accumulators, rounded up to a power of two
+    static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : (2 * BN <= 256 ? 256 : 512);
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+};
+
+__device__ __forceinline__ void unit_coords(const GemmArgs& g, int u, int& mb, int& nb,
+                                            int& split) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    split = u / tiles;
+    const int t = u - split * tiles;
+    const int per_group = kGroupM * g.num_n_blocks;
+    const int group = t / per_group;
+    const int first_m = group * kGroupM;
+    const int rem_m = g.num_m_blocks - first_m;
+    const int gm = rem_m < kGroupM ? rem_m : kGroupM;
+    const int idx = t - group * per_group;
+    mb = first_m + idx % gm;
+    nb = idx / gm;
+}
+
+__device__ __forceinline__ float gelu_f32(float x) {
+    return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
+}
+
+__device__ __forceinline__ float gelu_grad_f32(float x) {
+    const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
+    const float pdf = 0.39894228040143268f * expf(-0.5f * x * x);
+    return cdf + x * pdf;
+}
+
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+}
+
+__device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
+    const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float2 t = __bfloat1622float2(p[i]);
+        f[2 * i] = t.x;
+        f[2 * i + 1] = t.y;
+    }
+}
+
+// Epilogue of one 32-column chunk of one row: `acc` are the fp32
+// accumulators of columns col0 .. col0+31 of row `row`.
+template <int EPI>
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t (&acc)[32], int row,
+                                               int col0, int split) {
+    if (row >= g.M) return;
+    const int64_t off = static_cast<int64_t>(row) * g.ld_out + col0;
+    if constexpr (EPI == EPI_F32) {
+        float* out = static_cast<float*>(g.out0) + static_cast<int64_t>(split) * g.split_stride + off;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            if (col0 + 4 * q < g.N) {
+                float4 v = make_float4(__uint_as_float(acc[4 * q]), __uint_as_float(acc[4 * q + 1]),
+                                       __uint_as_float(acc[4 * q + 2]), __uint_as_float(acc[4 * q + 3]));
+                *reinterpret_cast<float4*>(out + 4 * q) = v;
+            }
+        }
+    } else {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const int c = col0 + 8 * q;
+            if (c >= g.N) continue;
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[8 * q + i]);
+            if constexpr (EPI == EPI_GELU || EPI == EPI_BIAS) {
+                if (g.bias != nullptr) {
+                    float bb[8];
+                    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.bias + c)), bb);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) v[i] += bb[i];
+                }
+            }
+            uint4 o0;
+            if constexpr (EPI == EPI_DGELU) {
+                float hh[8];
+                unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f32(hh[i]);
+            }
+            o0.x = pack_bf16x2(v[0], v[1]);
+            o0.y = pack_bf16x2(v[2], v[3]);
+            o0.z = pack_bf16x2(v[4], v[5]);
+            o0.w = pack_bf16x2(v[6], v[7]);
+            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off + 8 * q) = o0;
+            if constexpr (EPI == EPI_GELU) {
+                uint4 o1;
+                o1.x = pack_bf16x2(gelu_f32(v[0]), gelu_f32(v[1]));
+                o1.y = pack_bf16x2(gelu_f32(v[2]), gelu_f32(v[3]));
+                o1.z = pack_bf16x2(gelu_f32(v[4]), gelu_f32(v[5]));
+                o1.w = pack_bf16x2(gelu_f32(v[6]), gelu_f32(v[7]));
+                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out1) + off + 8 * q) = o1;
+            }
+        }
+    }
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const GemmArgs g) {
+    using C = TileCfg<BN>;
+    constexpr int STAGES = C::STAGES;
+    constexpr uint32_t IDESC = idesc_bf16_f32(kBM, BN, A_MN, B_MN);
+
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                               ~static_cast<uintptr_t>(1023));
+    uint8_t* sA = smem;
+    uint8_t* sB = smem + STAGES * C::A_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+    uint64_t* full = bars;
+    uint64_t* empty = bars + STAGES;
+    uint64_t* tfull = bars + 2 * STAGES;
+    uint64_t* tempty = bars + 2 * STAGES + 2;
+    uint64_t* drain = bars + 2 * STAGES + 4;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_u32(&full[s]), 1);
+            mbar_init(smem_u32(&empty[s]), 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(smem_u32(&tfull[b]), 1);
+            mbar_init(smem_u32(&tempty[b]), kEpiWarps);
+        }
+        mbar_init(smem_u32(drain), 1);
+        *abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem_base = *tmem_slot;
+
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    const int units = tiles * g.splits;
+    const uint64_t limit = g.wait_limit_ns;
+
+    if (warp == 0) {
+        // ------------------------------------------------ TMA producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmA);
+            tma_prefetch_desc(&tmB);
+            int stage = 0;
+            uint32_t phase = 0;
+            int issued = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
+                int mb, nb, split;
+                unit_coords(g, u, mb, nb, split);
+                const int kb0 = split * g.kb_per_split;
+                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort, limit)) {
+                        raise_timeout(abort);
+                        ok = false;
+                        break;
+                    }
+                    const uint32_t fb = smem_u32(&full[stage]);
+                    mbar_arrive_expect_tx(fb, C::STAGE_BYTES);
+                    const uint32_t a_dst = smem_u32(sA + stage * C::A_BYTES);
+                    const uint32_t b_dst = smem_u32(sB + stage * C::B_BYTES);
+                    if constexpr (!A_MN) {
+                        tma_load_2d(a_dst, &tmA, fb, kb * kBK, mb * kBM);
+                    } else {
+                        tma_load_2d(a_dst, &tmA, fb, mb * kBM, kb * kBK);
+                        tma_load_2d(a_dst + 8192, &tmA, fb, mb * kBM + 64, kb * kBK);
+                    }
+                    if constexpr (!B_MN) {
+                        tma_load_2d(b_dst, &tmB, fb, kb * kBK, nb * BN);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < BN / 64; ++j)
+                            tma_load_2d(b_dst + j * 8192, &tmB, fb, nb * BN + j * 64, kb * kBK);
+                    }
+                    ++issued;
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+            }
+            if (ok && !*abort) {
+                // Producer tail: wait until the MMA thread has released every
+                // slot, so no tensor-core completion is still due to arrive on
+                // this CTA's barriers when it exits.
+                int s = stage;
+                uint32_t ph = phase;
+                for (int i = 0; i < STAGES && ok; ++i) {
+                    if (!mbar_wait_bounded(smem_u32(&empty[s]), ph ^ 1u, abort, limit)) {
+                        raise_timeout(abort);
+                        ok = false;
+                    }
+                    if (++s == STAGES) {
+                        s = 0;
+                        ph ^= 1u;
+                    }
+                }
+            }
+            if (!ok || *abort) {
+                // Wind down: wait (bounded) for the copies still in flight, the
+                // most recent load of each of the last min(issued, STAGES) slots.
+                int s = stage;
+                uint32_t ph = phase;
+                const int n = issued < STAGES ? issued : STAGES;
+                for (int i = 0; i < n; ++i) {
+                    if (--s < 0) {
+                        s = STAGES - 1;
+                        ph ^= 1u;
+                    }
+                    volatile int never = 0;
+                    mbar_wait_bounded(smem_u32(&full[s]), ph, &never, limit);
+                }
+            }
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ------------------------------------------------ MMA issuer
+        if (lane == 0) {
+            int stage = 0;
+            uint32_t phase = 0;
+            int local = 0;
+            bool ok = true;
+            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++local) {
+                int mb, nb, split;
+                unit_coords(g, u, mb, nb, split);
+                const int kb0 = split * g.kb_per_split;
+                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
+                const int buf = local & 1;
+                const uint32_t aphase = (local >> 1) & 1;
+                if (!mbar_wait_bounded(smem_u32(&tempty[buf]), aphase ^ 1u, abort, limit)) {
+                    raise_timeout(abort);
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t d_tmem = tmem_base + static_cast<uint32_t>(buf * BN);
+                for (int kb = kb0; kb < kb1; ++kb) {
+                    if (!mbar_wait_bounded(smem_u32(&full[stage]), phase, abort, limit)) {
+                        raise_timeout(abort);
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t a_base = smem_u32(sA + stage * C::A_BYTES);
+                    const uint32_t b_base = smem_u32(sB + stage * C::B_BYTES);
+#pragma unroll
+                    for (int k = 0; k < kBK / 16; ++k) {
+                        // K-major: the 16-element k slice is 32 bytes further along
+                        // each 128-byte swizzled row. MN-major: it is 16 rows of
+                        // 128 bytes further down; 64-wide MN chunks are 8 KB apart.
+                        const uint64_t ad = A_MN ? smem_desc_sw128(a_base + k * 2048, 8192, 1024)
+                                                 : smem_desc_sw128(a_base + k * 32, 16, 1024);
+                        const uint64_t bd = B_MN ? smem_desc_sw128(b_base + k * 2048, 8192, 1024)
+                                                 : smem_desc_sw128(b_base + k * 32, 16, 1024);
+                        umma_bf16(d_tmem, ad, bd, IDESC, (kb > kb0 || k > 0) ? 1u : 0u);
+                    }
+                    umma_commit(smem_u32(&empty[stage]));
+                    if (++stage == STAGES) {
+                        stage = 0;
+                        phase ^= 1u;
+                    }
+                }
+                if (!ok) break;
+                umma_commit(smem_u32(&tfull[buf]));
+            }
+            if (!ok || *abort) {
+                // Wind down: wait (bounded) for every MMA issued so far.
+                umma_commit(smem_u32(drain));
+                volatile int never = 0;
+                mbar_wait_bounded(smem_u32(drain), 0, &never, limit);
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------ epilogue warps
+        const int quad = warp & 3;  // tensor-memory lanes this warp may access
+        int local = 0;
+        for (int u = blockIdx.x; u < units; u += gridDim.x, ++local) {
+            int mb, nb, split;
+            unit_coords(g, u, mb, nb, split);
+            const int buf = local & 1;
+            const uint32_t aphase = (local >> 1) & 1;
+            // every lane waits; the warp proceeds only if all lanes saw the
+            // phase complete, so the .sync.aligned loads below never diverge
+            const bool ok = mbar_wait_bounded(smem_u32(&tfull[buf]), aphase, abort, limit);
+            if (!__all_sync(0xffffffffu, ok)) {
+                raise_timeout(abort);
+                break;
+            }
+            tc_fence_after();
+            const int row = mb * kBM + quad * 32 + lane;
+            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                                   static_cast<uint32_t>(buf * BN);
+#pragma unroll 1
+            for (int c = 0; c < BN / 32; ++c) {
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(t_row + c * 32, acc);
+                tmem_wait_ld();
+                if (c == BN / 32 - 1) {
+                    // the whole accumulator is in registers: release it to the MMA warp
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
+                }
+                epilogue_chunk<EPI>(g, acc, row, nb * BN + c * 32, split);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem_base, C::TMEM_COLS);
+    }
+}
+
+}  // namespace tpmlp

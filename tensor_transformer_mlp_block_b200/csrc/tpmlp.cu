@@ -1,0 +1,622 @@
+// C ABI of the tensor-parallel MLP block: argument checks, planning and
+// kernel launches. See include/tpmlp.h for the contract of each entry point.
+//
+// The forward runs two GEMMs (page "Megatron", section "张量并行 / 数学原理"):
+//   F1  column-parallel  H, Y = X·A + a, GeLU(·)   output tiles never straddle
+//                        the shard boundary's meaning: every column of H is
+//                        independent, so shards are just column ranges
+//   F2  row-parallel     Z = Σ_i Y_i·B_i + b       the K loop runs over the
+//                        shards in ascending order (in tensor memory), or,
+//                        when the output tiles cannot fill the GPU, each
+//                        shard group writes an fp32 partial and the partials
+//                        are added in ascending order before the bias
+// and the backward four GEMMs plus two column sums (chain rule):
+//   B2  dH = (dZ·Bᵀ) ⊙ GeLU′(H)   B3  dB = Yᵀ·dZ   B4  dA = Xᵀ·dH
+//   B5  dX = Σ_i dH_i·A_iᵀ (ordered shard sum, as F2)   db, da column sums.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/tpmlp.h"
+#include "aux_kernels.cuh"
+#include "gemm_tc.cuh"
+#include "simt.cuh"
+
+namespace tpmlp {
+namespace {
+
+constexpr uint64_t kDefaultWaitLimitNs = 2000000000ull;
+constexpr int64_t kColsumRowsPerChunk = 128;
+constexpr int kMaxDevices = 64;
+
+std::atomic<uint64_t> g_launches{0};
+std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
+std::atomic<int> g_split_policy{0};
+
+struct DeviceInfo {
+    bool init = false;
+    int cc_major = 0;
+    int num_sms = 0;
+    uint32_t attr_set = 0;  // bit per tensor-core kernel instantiation
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mutex;
+
+const DeviceInfo* device_info() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_dev_mutex);
+    DeviceInfo& d = g_dev[dev];
+    if (!d.init) {
+        if (cudaDeviceGetAttribute(&d.cc_major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+            return nullptr;
+        if (cudaDeviceGetAttribute(&d.num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return nullptr;
+        d.init = true;
+    }
+    return &d;
+}
+
+// --------------------------------------------------------------- tensor maps
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Row-major bf16 matrix with `rows` rows of `cols` elements, read in boxes
+// of box_rows × 64 columns with the 128-byte swizzle (64 bf16 = 128 bytes).
+// Out-of-range box elements read as zero.
+bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int box_rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 2};
+    cuuint32_t box[2] = {64u, static_cast<cuuint32_t>(box_rows)};
+    cuuint32_t estr[2] = {1u, 1u};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+tpmlp_status check_launch() {
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? TPMLP_OK : TPMLP_ERR_CUDA;
+}
+
+// ------------------------------------------------------- per-kernel timing
+
+enum Kind : int {
+    K_F1 = 0, K_F2, K_F2_RED, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_B5_RED, K_MISC, K_COUNT
+};
+const char* const kKindNames[K_COUNT] = {
+    "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "F2.split_reduce", "B1.db_colsum",
+    "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
+    "B5.dgrad_dX_shard_sum", "B5.split_reduce",       "misc",
+};
+
+struct KindTotals {
+    uint64_t launches = 0;
+    double ms = 0, flops = 0, bytes = 0;
+};
+struct PendingRec {
+    cudaEvent_t a, b;
+    int kind;
+    double flops, bytes;
+};
+bool g_prof_on = false;
+KindTotals g_prof[K_COUNT];
+std::vector<PendingRec> g_pending;
+std::vector<cudaEvent_t> g_event_pool;
+
+cudaEvent_t pool_event() {
+    if (!g_event_pool.empty()) {
+        cudaEvent_t e = g_event_pool.back();
+        g_event_pool.pop_back();
+        return e;
+    }
+    cudaEvent_t e = nullptr;
+    cudaEventCreate(&e);
+    return e;
+}
+
+// Run `fn` (which enqueues one step's kernels on `st`); when timing is on,
+// bracket it with two events and remember the step's algorithmic work.
+template <class Fn>
+tpmlp_status timed(int kind, double flops, double bytes, cudaStream_t st, Fn&& fn) {
+    if (!g_prof_on) return fn();
+    cudaEvent_t a = pool_event(), b = pool_event();
+    if (a == nullptr || b == nullptr) return TPMLP_ERR_CUDA;
+    cudaEventRecord(a, st);
+    tpmlp_status s = fn();
+    cudaEventRecord(b, st);
+    g_pending.push_back({a, b, kind, flops, bytes});
+    return s;
+}
+
+// ------------------------------------------------------ tensor-core launches
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+constexpr int kernel_id() {
+    return (EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) + (BN == 128 ? 16 : 0);
+}
+
+// D[M, N] = Aop·Bop with Aop stored [M][K] (A_MN = false) or [K][M], Bop
+// stored [N][K] (B_MN = false) or [K][N]. `splits` > 1 splits the k-blocks
+// into equal consecutive ranges (EPI_F32 writes one plane per split).
+template <int BN, bool A_MN, bool B_MN, int EPI>
+tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int K, int splits,
+                            GemmArgs g, cudaStream_t st) {
+    using Cfg = TileCfg<BN>;
+    const DeviceInfo* dev = device_info();
+    if (dev == nullptr) return TPMLP_ERR_CUDA;
+    CUtensorMap tmA, tmB;
+    const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
+    const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN);
+    if (!okA || !okB) return TPMLP_ERR_CUDA;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.num_m_blocks = (M + kBM - 1) / kBM;
+    g.num_n_blocks = (N + BN - 1) / BN;
+    g.k_blocks = (K + kBK - 1) / kBK;
+    g.splits = splits;
+    g.kb_per_split = (g.k_blocks + splits - 1) / splits;
+    g.wait_limit_ns = g_wait_limit_ns.load();
+    auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI>;
+    constexpr int id = kernel_id<BN, A_MN, B_MN, EPI>();
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        int devn = 0;
+        cudaGetDevice(&devn);
+        if (!(g_dev[devn].attr_set & (1u << id))) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM_BYTES) != cudaSuccess)
+                return TPMLP_ERR_CUDA;
+            g_dev[devn].attr_set |= 1u << id;
+        }
+    }
+    const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
+    const int grid = static_cast<int>(units < dev->num_sms ? units : dev->num_sms);
+    kern<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, g);
+    return check_launch();
+}
+
+// Algorithmic bytes of one GEMM: both operands read once (bf16), the
+// outputs written once, plus the epilogue's extra input (saved H) and the
+// second output (Y) where the epilogue has them.
+template <int EPI>
+double gemm_bytes(double M, double N, double K, int splits) {
+    double b = 2.0 * (M * K + K * N);
+    if (EPI == EPI_GELU) b += 2.0 * 2.0 * M * N;
+    if (EPI == EPI_BIAS) b += 2.0 * M * N;
+    if (EPI == EPI_DGELU) b += 2.0 * 2.0 * M * N;
+    if (EPI == EPI_F32) b += 4.0 * M * N * splits;
+    return b;
+}
+
+template <int BN, bool A_MN, bool B_MN, int EPI>
+tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K, int splits,
+                     GemmArgs g, cudaStream_t st) {
+    return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K, splits), st, [&] {
+        return gemm_tc_launch<BN, A_MN, B_MN, EPI>(Aop, Bop, M, N, K, splits, g, st);
+    });
+}
+
+template <typename T, int EPI>
+tpmlp_status gemm_simt(int kind, const SimtArgs& a, cudaStream_t st) {
+    const double flops = 2.0 * a.M * a.N * a.K;
+    const double bytes = sizeof(T) * (1.0 * a.M * a.K + 1.0 * a.K * a.N) +
+                         (EPI == EPI_F32 ? 4.0 : sizeof(T) * (EPI == EPI_BIAS ? 1.0 : 2.0)) * a.M * a.N;
+    return timed(kind, flops, bytes, st, [&] {
+        dim3 grid((a.N + 15) / 16, (a.M + 15) / 16);
+        simt_gemm_kernel<T, EPI><<<grid, 256, 0, st>>>(a);
+        return check_launch();
+    });
+}
+
+// ---------------------------------------------------------------- planning
+
+struct Plan {
+    bool tc = false;    // tensor-core path (bf16, h % 8 == 0, F % 8 == 0)
+    int splits = 1;     // shard groups of the two row-parallel products
+    int64_t chunks = 1; // column-sum row chunks
+    size_t off_split = 0, off_cs_h = 0, off_cs_f = 0, total = 0;
+};
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+int choose_splits(int64_t T, int64_t h, int64_t F, int p, int num_sms) {
+    const int64_t Fp = F / p;
+    if (p == 1 || Fp % kBK != 0) return 1;
+    const int policy = g_split_policy.load();
+    if (policy == 1) return 1;
+    if (policy == 2) return p;
+    const int64_t tiles = ((T + kBM - 1) / kBM) * ((h + 255) / 256);
+    int S = 1;
+    while (S < p && tiles * S < num_sms) {
+        int next = S + 1;
+        while (p % next != 0) ++next;
+        S = next;
+    }
+    return S;
+}
+
+bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl) {
+    if (T < 0 || h < 1 || F < 1 || p < 1 || F % p != 0) return false;
+    if (dt != TPMLP_BF16 && dt != TPMLP_FP32) return false;
+    pl->tc = (dt == TPMLP_BF16) && (h % 8 == 0) && (F % 8 == 0);
+    int num_sms = 148;
+    if (const DeviceInfo* d = device_info()) num_sms = d->num_sms;
+    pl->splits = pl->tc ? choose_splits(T, h, F, p, num_sms) : 1;
+    pl->chunks = T > 0 ? (T + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk : 1;
+    size_t off = 0;
+    pl->off_split = off;
+    if (pl->splits > 1) off += round256(static_cast<size_t>(pl->splits) * T * h * sizeof(float));
+    pl->off_cs_h = off;
+    off += round256(static_cast<size_t>(pl->chunks) * h * sizeof(float));
+    pl->off_cs_f = off;
+    off += round256(static_cast<size_t>(pl->chunks) * F * sizeof(float));
+    pl->total = off;
+    return true;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+template <typename T>
+tpmlp_status colsum_launch(const T* X, int64_t R, int64_t C, int64_t chunks, float* partial,
+                           float* out, cudaStream_t st) {
+    dim3 grid(static_cast<unsigned>((C + 255) / 256), static_cast<unsigned>(chunks));
+    dim3 block(32, 8);
+    if (C % 8 == 0 && aligned16(X))
+        colsum_partial_kernel<T, true><<<grid, block, 0, st>>>(X, R, C, kColsumRowsPerChunk, partial);
+    else
+        colsum_partial_kernel<T, false><<<grid, block, 0, st>>>(X, R, C, kColsumRowsPerChunk, partial);
+    tpmlp_status s = check_launch();
+    if (s != TPMLP_OK) return s;
+    colsum_final_kernel<<<static_cast<unsigned>((C + 255) / 256), 256, 0, st>>>(
+        partial, static_cast<int>(chunks), C, out);
+    return check_launch();
+}
+
+// out = 1ᵀ·X for X: R × C; algorithmic bytes = X read once + out written.
+template <typename T>
+tpmlp_status colsum(int kind, const T* X, int64_t R, int64_t C, int64_t chunks, float* partial,
+                    float* out, cudaStream_t st) {
+    return timed(kind, 0.0, sizeof(T) * double(R) * C + 4.0 * C, st,
+                 [&] { return colsum_launch(X, R, C, chunks, partial, out, st); });
+}
+
+tpmlp_status reduce_splits_launch(const float* ws, int splits, int64_t M, int64_t N,
+                                  const void* bias, void* out, cudaStream_t st) {
+    const DeviceInfo* dev = device_info();
+    const int64_t groups = M * (N / 8);
+    int64_t blocks = (groups + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(dev ? dev->num_sms : 148) * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+    reduce_splits_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+        ws, splits, M * N, static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(out),
+        M, N);
+    return check_launch();
+}
+
+tpmlp_status reduce_splits(int kind, const float* ws, int splits, int64_t M, int64_t N,
+                           const void* bias, void* out, cudaStream_t st) {
+    return timed(kind, 0.0, 4.0 * splits * double(M) * N + 2.0 * double(M) * N, st,
+                 [&] { return reduce_splits_launch(ws, splits, M, N, bias, out, st); });
+}
+
+tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st) {
+    if (n <= 0) return TPMLP_OK;
+    return timed(K_MISC, 0.0, 4.0 * n, st, [&] {
+        int64_t blocks = (n + 255) / 256;
+        if (blocks > 1184) blocks = 1184;
+        zero_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, n);
+        return check_launch();
+    });
+}
+
+#define TPMLP_TRY(expr)                         \
+    do {                                        \
+        tpmlp_status _s = (expr);               \
+        if (_s != TPMLP_OK) return _s;          \
+    } while (0)
+
+tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl,
+                           void* ws, size_t ws_bytes) {
+    if (!make_plan(T, h, F, p, dt, pl)) return TPMLP_ERR_INVALID;
+    // the kernels index rows, columns and tiles with 32-bit integers
+    if (T >= (int64_t(1) << 31) || h >= (int64_t(1) << 31) || F >= (int64_t(1) << 31))
+        return TPMLP_ERR_UNSUPPORTED;
+    const DeviceInfo* d = device_info();
+    if (d == nullptr) return TPMLP_ERR_CUDA;
+    if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
+    if (pl->total > 0 && (ws == nullptr || ws_bytes < pl->total)) return TPMLP_ERR_WORKSPACE;
+    if (ws != nullptr && !aligned16(ws)) return TPMLP_ERR_ALIGN;
+    return TPMLP_OK;
+}
+
+}  // namespace
+}  // namespace tpmlp
+
+using namespace tpmlp;
+
+extern "C" {
+
+size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt) {
+    Plan pl;
+    if (!make_plan(T, h, F, p, dt, &pl)) return 0;
+    return pl.total;
+}
+
+tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void* B, const void* b,
+                        void* H, void* Y, void* Z, int64_t T, int64_t h, int64_t F, int p,
+                        tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+    cudaGetLastError();  // start from a clean (non-sticky) error state
+    Plan pl;
+    TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes));
+    if (T == 0) return TPMLP_OK;
+    if (!X || !A || !B || !H || !Y || !Z) return TPMLP_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (pl.tc) {
+        for (const void* q : {X, A, a, B, b, static_cast<const void*>(H), static_cast<const void*>(Y),
+                              static_cast<const void*>(Z)})
+            if (q && !aligned16(q)) return TPMLP_ERR_ALIGN;
+        const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
+        // F1: H = X·A + a, Y = GeLU(H). Aop = X [T][h] (K-major), Bop = A [h][F] (MN-major).
+        GemmArgs g1{};
+        g1.out0 = H;
+        g1.out1 = Y;
+        g1.ld_out = F;
+        g1.bias = static_cast<const __nv_bfloat16*>(a);
+        TPMLP_TRY((gemm_tc<256, false, true, EPI_GELU>(K_F1, X, A, iT, iF, ih, 1, g1, st)));
+        // F2: Z = Σ_i Y_i·B_i + b. Aop = Y [T][F] (K-major), Bop = B [F][h] (MN-major).
+        GemmArgs g2{};
+        if (pl.splits == 1) {
+            g2.out0 = Z;
+            g2.ld_out = h;
+            g2.bias = static_cast<const __nv_bfloat16*>(b);
+            TPMLP_TRY((gemm_tc<256, false, true, EPI_BIAS>(K_F2, Y, B, iT, ih, iF, 1, g2, st)));
+        } else {
+            float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
+            g2.out0 = ws;
+            g2.ld_out = h;
+            g2.split_stride = T * h;
+            TPMLP_TRY((gemm_tc<256, false, true, EPI_F32>(K_F2, Y, B, iT, ih, iF, pl.splits, g2, st)));
+            TPMLP_TRY(reduce_splits(K_F2_RED, ws, pl.splits, T, h, b, Z, st));
+        }
+        return TPMLP_OK;
+    }
+    // plain CUDA-core path: fp32, or bf16 with h or F not a multiple of 8
+    SimtArgs s1{};
+    s1.M = static_cast<int>(T); s1.N = static_cast<int>(F); s1.K = static_cast<int>(h);
+    s1.A = X; s1.sam = h; s1.sak = 1;
+    s1.B = A; s1.sbk = F; s1.sbn = 1;
+    s1.out0 = H; s1.out1 = Y; s1.ld_out = F; s1.bias = a;
+    SimtArgs s2{};
+    s2.M = static_cast<int>(T); s2.N = static_cast<int>(h); s2.K = static_cast<int>(F);
+    s2.A = Y; s2.sam = F; s2.sak = 1;
+    s2.B = B; s2.sbk = h; s2.sbn = 1;
+    s2.out0 = Z; s2.ld_out = h; s2.bias = b;
+    if (dt == TPMLP_FP32) {
+        TPMLP_TRY((gemm_simt<float, EPI_GELU>(K_F1, s1, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_F2, s2, st)));
+    } else {
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_GELU>(K_F1, s1, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_F2, s2, st)));
+    }
+    return TPMLP_OK;
+}
+
+tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void* B, const void* H,
+                        const void* Y, void* dX, float* dA, float* da, float* dB, float* db,
+                        void* dH, int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    cudaGetLastError();
+    Plan pl;
+    TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes));
+    if (!dA || !da || !dB || !db) return TPMLP_ERR_INVALID;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        TPMLP_TRY(zero_f32(dA, h * F, st));
+        TPMLP_TRY(zero_f32(da, F, st));
+        TPMLP_TRY(zero_f32(dB, F * h, st));
+        TPMLP_TRY(zero_f32(db, h, st));
+        return TPMLP_OK;
+    }
+    if (!dZ || !X || !A || !B || !H || !Y || !dX || !dH) return TPMLP_ERR_INVALID;
+    float* cs_h = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cs_h);
+    float* cs_f = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cs_f);
+    if (pl.tc) {
+        for (const void* q : {dZ, X, A, B, H, Y, static_cast<const void*>(dX),
+                              static_cast<const void*>(dA), static_cast<const void*>(da),
+                              static_cast<const void*>(dB), static_cast<const void*>(db),
+                              static_cast<const void*>(dH)})
+            if (!aligned16(q)) return TPMLP_ERR_ALIGN;
+        const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
+        const __nv_bfloat16* dZb = static_cast<const __nv_bfloat16*>(dZ);
+        // db = 1ᵀ·dZ
+        TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
+        // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
+        GemmArgs g2{};
+        g2.out0 = dH;
+        g2.ld_out = F;
+        g2.aux = static_cast<const __nv_bfloat16*>(H);
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_DGELU>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
+        // da = 1ᵀ·dH
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
+        // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
+        GemmArgs g3{};
+        g3.out0 = dB;
+        g3.ld_out = h;
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, 1, g3, st)));
+        // B4: dA = Xᵀ·dH. Aop = X [T][h] (MN-major, M = h), Bop = dH [T][F] (MN-major).
+        GemmArgs g4{};
+        g4.out0 = dA;
+        g4.ld_out = F;
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, 1, g4, st)));
+        // B5: dX = Σ_i dH_i·A_iᵀ. Aop = dH [T][F] (K-major), Bop = A [h][F] (K-major).
+        GemmArgs g5{};
+        if (pl.splits == 1) {
+            g5.out0 = dX;
+            g5.ld_out = h;
+            TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, 1, g5, st)));
+        } else {
+            float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
+            g5.out0 = ws;
+            g5.ld_out = h;
+            g5.split_stride = T * h;
+            TPMLP_TRY((gemm_tc<256, false, false, EPI_F32>(K_B5, dH, A, iT, ih, iF, pl.splits, g5, st)));
+            TPMLP_TRY(reduce_splits(K_B5_RED, ws, pl.splits, T, h, nullptr, dX, st));
+        }
+        return TPMLP_OK;
+    }
+    const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
+    // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H): Aop(t, j) = dZ[t][j], Bop(j, f) = B[f][j]
+    SimtArgs s2{};
+    s2.M = iT; s2.N = iF; s2.K = ih;
+    s2.A = dZ; s2.sam = h; s2.sak = 1;
+    s2.B = B; s2.sbk = 1; s2.sbn = h;
+    s2.out0 = dH; s2.ld_out = F; s2.aux = H;
+    // B3: dB = Yᵀ·dZ: Aop(f, t) = Y[t][f], Bop(t, j) = dZ[t][j]
+    SimtArgs s3{};
+    s3.M = iF; s3.N = ih; s3.K = iT;
+    s3.A = Y; s3.sam = 1; s3.sak = F;
+    s3.B = dZ; s3.sbk = h; s3.sbn = 1;
+    s3.out0 = dB; s3.ld_out = h;
+    // B4: dA = Xᵀ·dH: Aop(k, t) = X[t][k], Bop(t, f) = dH[t][f]
+    SimtArgs s4{};
+    s4.M = ih; s4.N = iF; s4.K = iT;
+    s4.A = X; s4.sam = 1; s4.sak = h;
+    s4.B = dH; s4.sbk = F; s4.sbn = 1;
+    s4.out0 = dA; s4.ld_out = F;
+    // B5: dX = dH·Aᵀ: Aop(t, f) = dH[t][f], Bop(f, k) = A[k][f]
+    SimtArgs s5{};
+    s5.M = iT; s5.N = ih; s5.K = iF;
+    s5.A = dH; s5.sam = F; s5.sak = 1;
+    s5.B = A; s5.sbk = 1; s5.sbn = F;
+    s5.out0 = dX; s5.ld_out = h;
+    if (dt == TPMLP_FP32) {
+        TPMLP_TRY(colsum(K_B1_DB, static_cast<const float*>(dZ), T, h, pl.chunks, cs_h, db, st));
+        TPMLP_TRY((gemm_simt<float, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const float*>(dH), T, F, pl.chunks, cs_f, da, st));
+        TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B3, s3, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B4, s4, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_B5, s5, st)));
+    } else {
+        TPMLP_TRY(colsum(K_B1_DB, static_cast<const __nv_bfloat16*>(dZ), T, h, pl.chunks, cs_h, db, st));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B3, s3, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B4, s4, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_B5, s5, st)));
+    }
+    return TPMLP_OK;
+}
+
+const char* tpmlp_strerror(tpmlp_status s) {
+    switch (s) {
+        case TPMLP_OK: return "ok";
+        case TPMLP_ERR_INVALID: return "invalid argument (size, p, null pointer or dtype)";
+        case TPMLP_ERR_ALIGN: return "pointer not 16-byte aligned";
+        case TPMLP_ERR_UNSUPPORTED: return "unsupported device or size";
+        case TPMLP_ERR_WORKSPACE: return "workspace missing or too small";
+        case TPMLP_ERR_CUDA: return "CUDA runtime or launch error";
+        case TPMLP_ERR_TIMEOUT: return "a kernel gave up a bounded wait";
+    }
+    return "unknown status";
+}
+
+tpmlp_status tpmlp_last_device_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return TPMLP_ERR_CUDA;
+    unsigned int v = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return TPMLP_ERR_CUDA;
+    if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+        return TPMLP_ERR_CUDA;
+    return v == 0 ? TPMLP_OK : static_cast<tpmlp_status>(v);
+}
+
+tpmlp_status tpmlp_set_split_policy(int policy) {
+    if (policy < 0 || policy > 2) return TPMLP_ERR_INVALID;
+    g_split_policy.store(policy);
+    return TPMLP_OK;
+}
+
+int tpmlp_get_split_policy(void) { return g_split_policy.load(); }
+
+void tpmlp_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns); }
+
+tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream) {
+    cudaGetLastError();
+    wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+    return check_launch();
+}
+
+uint64_t tpmlp_launch_count(void) { return g_launches.load(); }
+
+void tpmlp_profile_enable(int on) { g_prof_on = (on != 0); }
+
+int tpmlp_profile_collect(void) {
+    int rc = K_COUNT;
+    for (const PendingRec& r : g_pending) {
+        float ms = 0.0f;
+        if (cudaEventSynchronize(r.b) != cudaSuccess || cudaEventElapsedTime(&ms, r.a, r.b) != cudaSuccess) {
+            rc = -1;
+        } else {
+            KindTotals& t = g_prof[r.kind];
+            t.launches += 1;
+            t.ms += ms;
+            t.flops += r.flops;
+            t.bytes += r.bytes;
+        }
+        g_event_pool.push_back(r.a);
+        g_event_pool.push_back(r.b);
+    }
+    g_pending.clear();
+    return rc;
+}
+
+int tpmlp_profile_kinds(void) { return K_COUNT; }
+
+const char* tpmlp_profile_name(int kind) {
+    return (kind >= 0 && kind < K_COUNT) ? kKindNames[kind] : "unknown";
+}
+
+tpmlp_status tpmlp_profile_read(int kind, uint64_t* launches, double* total_ms, double* flops,
+                                double* bytes) {
+    if (kind < 0 || kind >= K_COUNT) return TPMLP_ERR_INVALID;
+    const KindTotals& t = g_prof[kind];
+    if (launches) *launches = t.launches;
+    if (total_ms) *total_ms = t.ms;
+    if (flops) *flops = t.flops;
+    if (bytes) *bytes = t.bytes;
+    return TPMLP_OK;
+}
+
+void tpmlp_profile_reset(void) {
+    for (KindTotals& t : g_prof) t = KindTotals{};
+}
+
+int tpmlp_version(void) { return 100; }
+
+}  // extern "C"

@@ -1,0 +1,110 @@
+"""The C ABI on the host: the library builds, loads and exports every entry
+point include/tpmlp.h declares; argument errors are reported before any
+launch (no GPU needed for these)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tpmlp.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from tensor_transformer_mlp_block_b200 import binding, build
+    build.build()
+    return binding.lib()
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"\b([a-z_][a-z0-9_]*)\s*\(", text)
+    return sorted({n for n in names if n.startswith(("tp_", "tpmlp_"))})
+
+
+def test_header_declares_expected_entry_points():
+    from tensor_transformer_mlp_block_b200 import binding
+    assert _declared_functions() == sorted(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    from tensor_transformer_mlp_block_b200 import build
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    out = subprocess.run(["nm", "-D", "--defined-only", build.LIB], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+
+
+def test_header_compiles_as_c(tmp_path):
+    src = tmp_path / "t.c"
+    src.write_text('#include "tpmlp.h"\nint main(void){ return (int)TPMLP_OK; }\n')
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    "-c", str(src), "-o", str(tmp_path / "t.o")], check=True)
+
+
+def test_strerror_covers_every_status(lib):
+    from tensor_transformer_mlp_block_b200 import binding
+    seen = set()
+    for s in range(7):
+        msg = binding.strerror(s)
+        assert msg and msg != "unknown status"
+        seen.add(msg)
+    assert len(seen) == 7
+    assert binding.strerror(99) == "unknown status"
+
+
+def test_version(lib):
+    assert lib.tpmlp_version() >= 100
+
+
+def test_invalid_arguments_fail_before_any_launch(lib):
+    from tensor_transformer_mlp_block_b200 import binding
+    before = binding.launch_count()
+    vp = ctypes.c_void_p(16)  # never dereferenced: validation fails first
+    cases = [
+        dict(T=8, h=8, F=16, p=0, dt=binding.BF16),   # p < 1
+        dict(T=8, h=8, F=16, p=3, dt=binding.BF16),   # F % p != 0
+        dict(T=-1, h=8, F=16, p=2, dt=binding.BF16),  # negative T
+        dict(T=8, h=0, F=16, p=2, dt=binding.BF16),   # h < 1
+        dict(T=8, h=8, F=16, p=2, dt=7),              # dtype code
+    ]
+    for c in cases:
+        st = lib.tp_mlp_fwd(vp, vp, None, vp, None, vp, vp, vp, c["T"], c["h"], c["F"], c["p"],
+                            c["dt"], None, 0, None)
+        assert st == binding.ERR_INVALID, c
+        st = lib.tp_mlp_bwd(vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, c["T"], c["h"], c["F"],
+                            c["p"], c["dt"], None, 0, None)
+        assert st == binding.ERR_INVALID, c
+    assert binding.launch_count() == before
+
+
+def test_workspace_size_host_logic(lib):
+    from tensor_transformer_mlp_block_b200 import binding
+    assert binding.workspace_size(8, 8, 16, 3) == 0  # invalid -> 0
+    binding.set_split_policy(1)
+    base = binding.workspace_size(1024, 512, 2048, 4)
+    binding.set_split_policy(2)
+    split = binding.workspace_size(1024, 512, 2048, 4)
+    binding.set_split_policy(0)
+    # forcing the shard split adds p fp32 planes of T×h
+    assert split - base >= 4 * 1024 * 512 * 4
+    assert base % 256 == 0 and split % 256 == 0
+    with pytest.raises(binding.TPMLPError):
+        binding.set_split_policy(3)
+
+
+def test_product_path_refuses_cpu_tensors():
+    import torch
+    from tensor_transformer_mlp_block_b200 import binding
+    X = torch.zeros(4, 8, dtype=torch.bfloat16)
+    A = torch.zeros(8, 16, dtype=torch.bfloat16)
+    B = torch.zeros(16, 8, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        binding.forward(X, A, None, B, None, 2)

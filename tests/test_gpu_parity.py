@@ -1,0 +1,136 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on
+the same seeded inputs, element by element.
+
+Small cases use the full oracle and span several 128×256 output tiles, a
+ragged K and ragged tails; the named workloads (GPT-2-small, 350M, 7B, 175B
+MLPs) are checked on seeded token rows and hidden columns that the oracle
+computes exactly, in the same launch configuration the bench times.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import TOL, compare_full, compare_sampled, oracle_full, rel_err, run_gpu, to_np
+from tensor_transformer_mlp_block_b200 import configs
+from tensor_transformer_mlp_block_b200.inputs import make_inputs, make_shape, sample_indices
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(autouse=True)
+def _auto_policy():
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(0)
+    yield
+    binding.set_split_policy(0)
+
+
+def test_tiny_fp32_full():
+    cfg = configs.get("tiny")
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p)
+    compare_full(gpu, oracle_full(inp), "fp32")
+
+
+@pytest.mark.parametrize("T,h,F,p", [
+    (300, 200, 520, 2),    # ragged M (2 tiles + 44 rows), ragged K (200), ragged N (520)
+    (256, 128, 512, 4),    # whole tiles, Fp = 128 (two k-blocks per shard)
+    (129, 64, 264, 3),     # one row past a tile, single k-block, Fp = 88
+    (1, 8, 8, 1),          # single token, smallest aligned shape
+    (640, 96, 776, 1),     # p = 1: the unsplit MLP
+])
+def test_bf16_full_oracle(T, h, F, p):
+    inp = make_shape(T, h, F, "bf16", seed_offset=T + h + F)
+    gpu = run_gpu(inp, p)
+    compare_full(gpu, oracle_full(inp), "bf16")
+
+
+def test_bf16_unaligned_shape_plain_path():
+    """h and F not multiples of 8: the plain CUDA-core kernels serve bf16."""
+    inp = make_shape(37, 12, 44, "bf16", seed_offset=9)
+    gpu = run_gpu(inp, 2)
+    compare_full(gpu, oracle_full(inp), "bf16")
+
+
+@pytest.mark.parametrize("policy", [1, 2])
+def test_row_parallel_split_policies(policy):
+    """Both schedules of the row-parallel products (shard K-loop in tensor
+    memory; per-shard fp32 partials summed in order) match the oracle."""
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(policy)
+    inp = make_shape(384, 320, 1024, "bf16", seed_offset=11)
+    gpu = run_gpu(inp, 4)
+    compare_full(gpu, oracle_full(inp), "bf16")
+
+
+def test_shard_count_invariance():
+    """p changes the partition, not the math: every p gives the oracle's
+    result, and any two p agree within the same bound."""
+    from tensor_transformer_mlp_block_b200 import binding
+    inp = make_shape(256, 256, 2048, "bf16", seed_offset=13)
+    ref = oracle_full(inp)
+    outs = {}
+    for policy in (1, 2):
+        binding.set_split_policy(policy)
+        for p in (1, 2, 4, 8):
+            outs[(policy, p)] = run_gpu(inp, p)
+            compare_full(outs[(policy, p)], ref, "bf16")
+    base = outs[(1, 1)]
+    for key, o in outs.items():
+        for k in ref:
+            rms = float(np.sqrt(np.mean(ref[k] ** 2)))
+            diff = float(np.max(np.abs(to_np(o[k]) - to_np(base[k]))))
+            assert diff <= TOL["bf16"] * rms, (key, k, diff / rms)
+
+
+def test_deterministic_bitwise():
+    inp = make_shape(300, 200, 520, "bf16", seed_offset=17)
+    a = run_gpu(inp, 2)
+    b = run_gpu(inp, 2)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_empty_tokens():
+    from tensor_transformer_mlp_block_b200 import binding
+    inp = make_shape(0, 64, 256, "bf16")
+    d = {k: v.cuda() for k, v in inp.items()}
+    H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], 2)
+    assert H.shape == (0, 256) and Z.shape == (0, 64)
+    out = dict(dX=torch.empty((0, 64), dtype=torch.bfloat16, device="cuda"),
+               dA=torch.full((64, 256), 7.0, device="cuda"), da=torch.full((256,), 7.0, device="cuda"),
+               dB=torch.full((256, 64), 7.0, device="cuda"), db=torch.full((64,), 7.0, device="cuda"),
+               dH=torch.empty((0, 256), dtype=torch.bfloat16, device="cuda"))
+    g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, 2, out=out)
+    for k in ("dA", "da", "dB", "db"):
+        assert torch.count_nonzero(g[k]).item() == 0, k
+
+
+def test_nan_propagates_without_fault():
+    from tensor_transformer_mlp_block_b200 import binding
+    inp = make_shape(256, 128, 512, "bf16", seed_offset=19)
+    inp["X"][5, 3] = float("nan")
+    gpu = run_gpu(inp, 2)
+    assert torch.isnan(gpu["Z"][5]).all()
+    assert not torch.isnan(gpu["Z"][6]).any()
+    assert binding.last_device_status() == 0
+
+
+@pytest.mark.parametrize("name", ["gpt2-small", "350m", "7b", "175b"])
+def test_named_config_sampled(name):
+    cfg = configs.get(name)
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p)
+    n_rows = 16 if name == "175b" else 48
+    R = sample_indices(cfg.T, n_rows, seed=1234).numpy()
+    J = sample_indices(cfg.F, 64, seed=1235).numpy()
+    errs = compare_sampled(gpu, inp, R, J, cfg.dtype)
+    assert all(np.isfinite(list(errs.values())))
+
+
+def test_named_config_gpt2_full():
+    """The GPT-2-small MLP against the full oracle (every element)."""
+    cfg = configs.get("gpt2-small")
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p)
+    compare_full(gpu, oracle_full(inp), "bf16")
