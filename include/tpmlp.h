@@ -151,6 +151,36 @@ tpmlp_status tpmlp_profile_read(int kind, uint64_t* launches, double* total_ms, 
                                 double* bytes);
 void tpmlp_profile_reset(void);
 
+/* Backward that allocates nothing and takes no workspace. The pages have no
+ * counterpart: this entry point exists for callers that cannot allocate
+ * device memory when they run the backward, such as a plugin inside another
+ * framework that owns all device allocations and offers extensions no
+ * allocator, or a runtime with a fixed memory budget that forbids
+ * allocation after start-up (cudaMalloc and cudaFree can also synchronize
+ * the device, which such callers must avoid).
+ * Computes exactly what tp_mlp_bwd computes, with the same arguments minus
+ * the workspace, and the same requirements. Its only scratch, the partial
+ * column sums of db and da, is a fixed 8 MiB array inside this library
+ * (tpmlp_noalloc_scratch_bytes()), held on every GPU that loads the library
+ * until the process exits; dX always uses the unsplit schedule (each output
+ * tile loops over the shards in ascending order), which needs no scratch.
+ * The call needs 4·ceil(T/128)·h + 4·ceil(T/128)·F bytes of it (each part
+ * rounded up to a multiple of 256); larger sizes return TPMLP_ERR_WORKSPACE
+ * before any launch. It calls no allocating routine.
+ * The first call on each device looks up the array's device address
+ * (cudaGetSymbolAddress) with that device current; make that first call
+ * before any stream capture. Every call shares the one array: calls whose
+ * kernels overlap on the GPU (on different streams or host threads) race on
+ * it and give undefined gradients. Nothing in the array needs to start at
+ * zero; each call writes every partial before reading it. */
+tpmlp_status tp_mlp_bwd_noalloc(const void* dZ, const void* X, const void* A, const void* B,
+                                const void* H, const void* Y, void* dX, float* dA, float* da,
+                                float* dB, float* db, void* dH, int64_t T, int64_t h, int64_t F,
+                                int p, tpmlp_dtype dt, void* stream);
+
+/* Size in bytes of the fixed scratch array tp_mlp_bwd_noalloc uses. */
+size_t tpmlp_noalloc_scratch_bytes(void);
+
 /* Library version, major·10000 + minor·100 + patch. */
 int tpmlp_version(void);
 

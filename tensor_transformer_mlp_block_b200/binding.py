@@ -24,7 +24,8 @@ EXPORTS = (
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
-    "tpmlp_profile_read", "tpmlp_profile_reset", "tpmlp_version",
+    "tpmlp_profile_read", "tpmlp_profile_reset", "tp_mlp_bwd_noalloc",
+    "tpmlp_noalloc_scratch_bytes", "tpmlp_version",
 )
 
 _lib = None
@@ -77,6 +78,9 @@ def lib() -> ctypes.CDLL:
                 [ctypes.POINTER(ctypes.c_double)] * 3
             L.tpmlp_profile_read.restype = ctypes.c_int
             L.tpmlp_profile_reset.restype = None
+            L.tp_mlp_bwd_noalloc.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp]
+            L.tp_mlp_bwd_noalloc.restype = ctypes.c_int
+            L.tpmlp_noalloc_scratch_bytes.restype = sz
             _lib = L
     return _lib
 

@@ -620,3 +620,153 @@ void tpmlp_profile_reset(void) {
 int tpmlp_version(void) { return 100; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward without any caller-provided memory beyond inputs and outputs.
+//
+// Some callers cannot allocate device memory when they call the backward:
+// a plugin running inside another framework that owns every device
+// allocation and gives its extensions no allocator, or a runtime with a
+// fixed memory budget that forbids allocation after start-up (cudaMalloc
+// and cudaFree may also synchronize the device, which such callers avoid).
+// tp_mlp_bwd_noalloc serves them: its only scratch, the partial column sums
+// of the two bias gradients, lives in a fixed array compiled into this
+// library, and it always uses the unsplit schedule for dX (each output tile
+// loops over the shards in ascending order in tensor memory), which needs
+// no scratch.
+namespace tpmlp {
+namespace {
+
+// 8 MiB, resident on every GPU that loads this library until the process
+// exits. The column-sum partials of a call need
+// 4·ceil(T/128)·h + 4·ceil(T/128)·F bytes (each part rounded up to 256).
+constexpr size_t kNoallocScratchBytes = size_t(8) << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoallocScratchBytes];
+
+// Device address of g_noalloc_scratch, per device. In host code the
+// array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device, with that device current.
+void* g_noalloc_ptr[kMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+tpmlp_status noalloc_scratch_ptr(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return TPMLP_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+            return TPMLP_ERR_CUDA;
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return TPMLP_OK;
+}
+
+}  // namespace
+}  // namespace tpmlp
+
+extern "C" {
+
+size_t tpmlp_noalloc_scratch_bytes(void) { return kNoallocScratchBytes; }
+
+tpmlp_status tp_mlp_bwd_noalloc(const void* dZ, const void* X, const void* A, const void* B,
+                                const void* H, const void* Y, void* dX, float* dA, float* da,
+                                float* dB, float* db, void* dH, int64_t T, int64_t h, int64_t F,
+                                int p, tpmlp_dtype dt, void* stream) {
+    cudaGetLastError();
+    Plan pl;
+    if (!make_plan(T, h, F, p, dt, &pl)) return TPMLP_ERR_INVALID;
+    if (T >= (int64_t(1) << 31) || h >= (int64_t(1) << 31) || F >= (int64_t(1) << 31))
+        return TPMLP_ERR_UNSUPPORTED;
+    const DeviceInfo* d = device_info();
+    if (d == nullptr) return TPMLP_ERR_CUDA;
+    if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
+    const size_t cs_h_bytes = round256(static_cast<size_t>(pl.chunks) * h * sizeof(float));
+    const size_t cs_f_bytes = round256(static_cast<size_t>(pl.chunks) * F * sizeof(float));
+    if (cs_h_bytes + cs_f_bytes > kNoallocScratchBytes) return TPMLP_ERR_WORKSPACE;
+    if (!dA || !da || !dB || !db) return TPMLP_ERR_INVALID;
+    if (T > 0 && (!dZ || !X || !A || !B || !H || !Y || !dX || !dH)) return TPMLP_ERR_INVALID;
+    if (pl.tc && T > 0) {
+        for (const void* q : {dZ, X, A, B, H, Y, static_cast<const void*>(dX),
+                              static_cast<const void*>(dA), static_cast<const void*>(da),
+                              static_cast<const void*>(dB), static_cast<const void*>(db),
+                              static_cast<const void*>(dH)})
+            if (!aligned16(q)) return TPMLP_ERR_ALIGN;
+    }
+    void* scratch = nullptr;
+    TPMLP_TRY(noalloc_scratch_ptr(&scratch));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (T == 0) {
+        TPMLP_TRY(zero_f32(dA, h * F, st));
+        TPMLP_TRY(zero_f32(da, F, st));
+        TPMLP_TRY(zero_f32(dB, F * h, st));
+        TPMLP_TRY(zero_f32(db, h, st));
+        return TPMLP_OK;
+    }
+    // Every partial the column sums use is written before it is read, so
+    // nothing in the scratch has to start at zero.
+    float* cs_h = static_cast<float*>(scratch);
+    float* cs_f = reinterpret_cast<float*>(static_cast<char*>(scratch) + cs_h_bytes);
+    const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
+    if (pl.tc) {
+        TPMLP_TRY(colsum(K_B1_DB, static_cast<const __nv_bfloat16*>(dZ), T, h, pl.chunks, cs_h, db, st));
+        GemmArgs g2{};
+        g2.out0 = dH;
+        g2.ld_out = F;
+        g2.aux = static_cast<const __nv_bfloat16*>(H);
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_DGELU>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
+        GemmArgs g3{};
+        g3.out0 = dB;
+        g3.ld_out = h;
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, 1, g3, st)));
+        GemmArgs g4{};
+        g4.out0 = dA;
+        g4.ld_out = F;
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, 1, g4, st)));
+        GemmArgs g5{};
+        g5.out0 = dX;
+        g5.ld_out = h;
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, 1, g5, st)));
+        return TPMLP_OK;
+    }
+    SimtArgs s2{};
+    s2.M = iT; s2.N = iF; s2.K = ih;
+    s2.A = dZ; s2.sam = h; s2.sak = 1;
+    s2.B = B; s2.sbk = 1; s2.sbn = h;
+    s2.out0 = dH; s2.ld_out = F; s2.aux = H;
+    SimtArgs s3{};
+    s3.M = iF; s3.N = ih; s3.K = iT;
+    s3.A = Y; s3.sam = 1; s3.sak = F;
+    s3.B = dZ; s3.sbk = h; s3.sbn = 1;
+    s3.out0 = dB; s3.ld_out = h;
+    SimtArgs s4{};
+    s4.M = ih; s4.N = iF; s4.K = iT;
+    s4.A = X; s4.sam = 1; s4.sak = h;
+    s4.B = dH; s4.sbk = F; s4.sbn = 1;
+    s4.out0 = dA; s4.ld_out = F;
+    SimtArgs s5{};
+    s5.M = iT; s5.N = ih; s5.K = iF;
+    s5.A = dH; s5.sam = F; s5.sak = 1;
+    s5.B = A; s5.sbk = 1; s5.sbn = F;
+    s5.out0 = dX; s5.ld_out = h;
+    if (dt == TPMLP_FP32) {
+        TPMLP_TRY(colsum(K_B1_DB, static_cast<const float*>(dZ), T, h, pl.chunks, cs_h, db, st));
+        TPMLP_TRY((gemm_simt<float, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const float*>(dH), T, F, pl.chunks, cs_f, da, st));
+        TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B3, s3, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B4, s4, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_B5, s5, st)));
+    } else {
+        TPMLP_TRY(colsum(K_B1_DB, static_cast<const __nv_bfloat16*>(dZ), T, h, pl.chunks, cs_h, db, st));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B3, s3, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B4, s4, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_B5, s5, st)));
+    }
+    return TPMLP_OK;
+}
+
+}  // extern "C"
