@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtpmlp.so")
 SOURCES = ["tpmlp.cu"]
-HEADERS = ["ptx.cuh", "gemm_tc.cuh", "aux_kernels.cuh", "simt.cuh"]
+HEADERS = ["ptx.cuh", "gemm_tc.cuh", "gemm_tc2.cuh", "aux_kernels.cuh", "simt.cuh"]
 INCLUDE = os.path.join(os.path.dirname(HERE), "include", "tpmlp.h")
 
 NVCC_FLAGS = [

@@ -25,6 +25,7 @@
 #include "../../include/tpmlp.h"
 #include "aux_kernels.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "simt.cuh"
 
 namespace tpmlp {
@@ -42,7 +43,9 @@ struct DeviceInfo {
     bool init = false;
     int cc_major = 0;
     int num_sms = 0;
-    uint32_t attr_set = 0;  // bit per tensor-core kernel instantiation
+    uint32_t attr_set = 0;       // bit per one-CTA tensor-core kernel instantiation
+    uint32_t attr_set_pair = 0;  // bit per CTA-pair kernel instantiation
+    int max_pairs[32] = {};      // co-resident CTA pairs per pair-kernel instantiation
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -201,6 +204,62 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     return check_launch();
 }
 
+// Same product on CTA pairs: 256 × BN tiles, grid = 2 × (co-resident pairs).
+template <int BN, bool A_MN, bool B_MN, int EPI>
+tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int K, int splits,
+                             GemmArgs g, cudaStream_t st) {
+    using Cfg = Tile2Cfg<BN>;
+    const DeviceInfo* dev = device_info();
+    if (dev == nullptr) return TPMLP_ERR_CUDA;
+    CUtensorMap tmA, tmB;
+    const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
+    const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN / 2);
+    if (!okA || !okB) return TPMLP_ERR_CUDA;
+    g.M = M;
+    g.N = N;
+    g.K = K;
+    g.num_m_blocks = (M + kPairM - 1) / kPairM;
+    g.num_n_blocks = (N + BN - 1) / BN;
+    g.k_blocks = (K + kBK - 1) / kBK;
+    g.splits = splits;
+    g.kb_per_split = (g.k_blocks + splits - 1) / splits;
+    g.wait_limit_ns = g_wait_limit_ns.load();
+    auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI>;
+    constexpr int id = kernel_id<BN, A_MN, B_MN, EPI>();
+    int max_pairs = 0;
+    {
+        std::lock_guard<std::mutex> lock(g_dev_mutex);
+        int devn = 0;
+        cudaGetDevice(&devn);
+        DeviceInfo& d = g_dev[devn];
+        if (!(d.attr_set_pair & (1u << id))) {
+            if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     Cfg::SMEM_BYTES) != cudaSuccess)
+                return TPMLP_ERR_CUDA;
+            cudaLaunchConfig_t cfg = {};
+            cfg.gridDim = dim3(static_cast<unsigned>(2 * (d.num_sms / 2)));
+            cfg.blockDim = dim3(kThreads);
+            cfg.dynamicSmemBytes = Cfg::SMEM_BYTES;
+            cudaLaunchAttribute attr;
+            attr.id = cudaLaunchAttributeClusterDimension;
+            attr.val.clusterDim.x = 2;
+            attr.val.clusterDim.y = 1;
+            attr.val.clusterDim.z = 1;
+            cfg.attrs = &attr;
+            cfg.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return TPMLP_ERR_CUDA;
+            d.max_pairs[id] = n;
+            d.attr_set_pair |= 1u << id;
+        }
+        max_pairs = d.max_pairs[id];
+    }
+    const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
+    const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
+    kern<<<2 * pairs, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, g);
+    return check_launch();
+}
+
 // Algorithmic bytes of one GEMM: both operands read once (bf16), the
 // outputs written once, plus the epilogue's extra input (saved H) and the
 // second output (Y) where the epilogue has them.
@@ -218,6 +277,8 @@ template <int BN, bool A_MN, bool B_MN, int EPI>
 tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K, int splits,
                      GemmArgs g, cudaStream_t st) {
     return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K, splits), st, [&] {
+        // CTA pairs whenever a 256-row tile is not mostly padding
+        if (M > kBM) return gemm_tc2_launch<BN, A_MN, B_MN, EPI>(Aop, Bop, M, N, K, splits, g, st);
         return gemm_tc_launch<BN, A_MN, B_MN, EPI>(Aop, Bop, M, N, K, splits, g, st);
     });
 }
