@@ -132,6 +132,18 @@ tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream);
 /* Number of kernels this library has launched in this process. */
 uint64_t tpmlp_launch_count(void);
 
+/* Evaluates GeLU(x[i]) into y[i] and GeLU′(x[i]) into dy[i] (fp32 device
+ * arrays of n elements) with one of the two forms the kernels use, so the
+ * approximation can be checked against CUDA's functions:
+ *   form 0: the tensor-core epilogues' form, Φ(x) from the rational erf
+ *           approximation of C. Hastings (Abramowitz & Stegun, Handbook of
+ *           Mathematical Functions, eq. 7.1.26, |error| ≤ 1.5e−7) sharing
+ *           exp(−x²/2) with φ(x);
+ *   form 1: the plain path's form through CUDA's erff and expf.
+ * Returns TPMLP_ERR_INVALID for n < 0, null pointers or another form. */
+tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t n, int form,
+                                   void* stream);
+
 /* Per-kernel timing on the launching stream, for measurement tools. While
  * enabled (on != 0), every kernel launch is bracketed by a pair of CUDA
  * events on its stream and tagged with its step (F1 column GEMM, F2 row

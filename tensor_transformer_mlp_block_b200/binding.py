@@ -22,7 +22,7 @@ BF16, FP32 = 0, 1
 EXPORTS = (
     "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
-    "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count",
+    "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
     "tpmlp_profile_read", "tpmlp_profile_reset", "tp_mlp_bwd_noalloc",
     "tpmlp_noalloc_scratch_bytes", "tpmlp_version",
@@ -67,6 +67,8 @@ def lib() -> ctypes.CDLL:
             L.tpmlp_wait_selftest.argtypes = [ctypes.c_uint64, vp]
             L.tpmlp_wait_selftest.restype = ctypes.c_int
             L.tpmlp_launch_count.restype = ctypes.c_uint64
+            L.tpmlp_eval_activation.argtypes = [vp, vp, vp, i64, ctypes.c_int, vp]
+            L.tpmlp_eval_activation.restype = ctypes.c_int
             L.tpmlp_version.restype = ctypes.c_int
             L.tpmlp_profile_enable.argtypes = [ctypes.c_int]
             L.tpmlp_profile_enable.restype = None
@@ -257,3 +259,16 @@ def profile_collect() -> dict:
             out[L.tpmlp_profile_name(k).decode()] = dict(launches=int(cnt.value), ms=ms.value,
                                                          flops=fl.value, bytes=by.value)
     return out
+
+
+def eval_activation(x: torch.Tensor, form: int):
+    """(GeLU(x), GeLU′(x)) of a CUDA fp32 tensor with the kernels' form 0
+    (Hastings erf, tensor-core epilogues) or 1 (CUDA erff, plain path)."""
+    if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous CUDA float32 tensor")
+    y = torch.empty_like(x)
+    dy = torch.empty_like(x)
+    _check(lib().tpmlp_eval_activation(x.data_ptr(), y.data_ptr(), dy.data_ptr(), x.numel(),
+                                       int(form), _stream_ptr(x.device, None)),
+           "tpmlp_eval_activation")
+    return y, dy

@@ -118,6 +118,18 @@ __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restri
     out[c] = s;
 }
 
+// GeLU and GeLU′ of n values with either form the library uses:
+// form 0 = the tensor-core epilogues' (Hastings erf), 1 = CUDA's erff/expf.
+__global__ void eval_activation_kernel(const float* __restrict__ x, float* __restrict__ y,
+                                       float* __restrict__ dy, int64_t n, int form) {
+    for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+         i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+        const float v = x[i];
+        y[i] = form == 0 ? gelu_fast(v) : gelu_f32(v);
+        dy[i] = form == 0 ? gelu_grad_fast(v) : gelu_grad_f32(v);
+    }
+}
+
 __global__ void zero_f32_kernel(float* __restrict__ p, int64_t n) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)

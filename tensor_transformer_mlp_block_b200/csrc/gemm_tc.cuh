@@ -52,9 +52,13 @@ struct GemmArgs {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kThreads = 192;
-constexpr int kEpiWarps = 4;
+constexpr int kEpiWarps = 8;  // two per SM sub-partition, each half of the columns
+constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kGroupM = 16;  // m-blocks per raster group (L2 reuse of Bop)
+// Shared-memory staging for the epilogue's bulk stores: one 4 KB slot per
+// epilogue warp (a 32 × 32 fp32 chunk, or two 32 × 32 bf16 chunks).
+constexpr int kEpiSlotBytes = 4096;
+constexpr int kEpiStagingBytes = kEpiWarps * kEpiSlotBytes;
 
 template <int BN>
 struct TileCfg {
@@ -66,7 +70,7 @@ struct TileCfg {
     // tensor-memory columns: two accumulators, rounded up to a power of two
     static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : (2 * BN <= 256 ? 256 : 512);
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
 __device__ __forceinline__ void unit_coords(const GemmArgs& g, int u, int& mb, int& nb,
@@ -84,6 +88,7 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& g, int u, int& mb, i
     nb = idx / gm;
 }
 
+// GeLU and its derivative through CUDA's erff/expf (the plain path).
 __device__ __forceinline__ float gelu_f32(float x) {
     return 0.5f * x * (1.0f + erff(x * 0.70710678118654752f));
 }
@@ -92,6 +97,39 @@ __device__ __forceinline__ float gelu_grad_f32(float x) {
     const float cdf = 0.5f * (1.0f + erff(x * 0.70710678118654752f));
     const float pdf = 0.39894228040143268f * expf(-0.5f * x * x);
     return cdf + x * pdf;
+}
+
+// Φ(x) and g = exp(−x²/2) for the tensor-core epilogues, from the rational
+// approximation of erf by C. Hastings as printed in Abramowitz & Stegun,
+// Handbook of Mathematical Functions, eq. 7.1.26:
+//   erf(z) = 1 − (a1·t + a2·t² + a3·t³ + a4·t⁴ + a5·t⁵)·exp(−z²),
+//   t = 1/(1 + p·z), z ≥ 0, |error| ≤ 1.5e−7.
+// With z = |x|/√2, exp(−z²) = exp(−x²/2) is the same factor the normal
+// density needs, so Φ and φ = g/√(2π) cost one exponential and one
+// reciprocal. Φ(−|x|) = ½·(1 − erf(z)); Φ(x) = 1 − Φ(−x).
+__device__ __forceinline__ void normal_cdf_and_gauss(float x, float& cdf, float& g) {
+    const float z = fabsf(x) * 0.70710678118654752f;
+    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
+    float poly = fmaf(1.061405429f, t, -1.453152027f);
+    poly = fmaf(poly, t, 1.421413741f);
+    poly = fmaf(poly, t, -0.284496736f);
+    poly = fmaf(poly, t, 0.254829592f);
+    poly *= t;
+    g = __expf(-0.5f * x * x);
+    const float tail = 0.5f * poly * g;  // Φ(−|x|)
+    cdf = x >= 0.0f ? 1.0f - tail : tail;
+}
+
+__device__ __forceinline__ float gelu_fast(float x) {
+    float cdf, g;
+    normal_cdf_and_gauss(x, cdf, g);
+    return x * cdf;
+}
+
+__device__ __forceinline__ float gelu_grad_fast(float x) {
+    float cdf, g;
+    normal_cdf_and_gauss(x, cdf, g);
+    return fmaf(x * 0.39894228040143268f, g, cdf);
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -109,59 +147,85 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
     }
 }
 
-// Epilogue of one 32-column chunk of one row: `acc` are the fp32
-// accumulators of columns col0 .. col0+31 of row `row`.
+// Epilogue of one 32 × 32 chunk of the accumulator: this warp's 32 rows
+// row0 .. row0+31 (lane i holds row row0 + i) and columns col0 .. col0+31.
+// The results are written row by row into the warp's shared-memory staging
+// slot in the swizzled layout the output tensor map expects (bf16: 64-byte
+// rows, 64-byte swizzle; fp32: 128-byte rows, 128-byte swizzle, which makes
+// the 16-byte shared stores of a warp bank-conflict free), then one lane
+// stores the whole chunk with a TMA bulk tensor store, which clips rows and
+// columns outside the output. The slot is reused only after the previous
+// store of this warp has finished reading it.
 template <int EPI>
-__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t (&acc)[32], int row,
-                                               int col0, int split) {
-    if (row >= g.M) return;
-    const int64_t off = static_cast<int64_t>(row) * g.ld_out + col0;
+__device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensorMap* tmO0,
+                                               const CUtensorMap* tmO1, const uint32_t (&acc)[32],
+                                               int row0, int col0, int split, uint32_t slot,
+                                               int lane) {
+    const int row = row0 + lane;
+    const bool any = (row0 < g.M) && (col0 < g.N);
     if constexpr (EPI == EPI_F32) {
-        float* out = static_cast<float*>(g.out0) + static_cast<int64_t>(split) * g.split_stride + off;
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (col0 + 4 * q < g.N) {
-                float4 v = make_float4(__uint_as_float(acc[4 * q]), __uint_as_float(acc[4 * q + 1]),
-                                       __uint_as_float(acc[4 * q + 2]), __uint_as_float(acc[4 * q + 3]));
-                *reinterpret_cast<float4*>(out + 4 * q) = v;
-            }
+        for (int j = 0; j < 8; ++j) {
+            uint4 v = make_uint4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]);
+            st_shared_v4(slot + lane * 128 + ((j ^ (lane & 7)) << 4), v);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && any) {
+            tma_store_3d(tmO0, slot, col0, row0, split);
+            bulk_commit();
         }
     } else {
+        uint4 o0[4], o1[4];
+        const int64_t off = static_cast<int64_t>(row) * g.ld_out + col0;
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int c = col0 + 8 * q;
-            if (c >= g.N) continue;
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[8 * q + i]);
             if constexpr (EPI == EPI_GELU || EPI == EPI_BIAS) {
-                if (g.bias != nullptr) {
+                if (g.bias != nullptr && c < g.N) {
                     float bb[8];
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.bias + c)), bb);
 #pragma unroll
                     for (int i = 0; i < 8; ++i) v[i] += bb[i];
                 }
             }
-            uint4 o0;
             if constexpr (EPI == EPI_DGELU) {
-                float hh[8];
-                unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
+                float hh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+                if (row < g.M && c < g.N)
+                    unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_f32(hh[i]);
+                for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_fast(hh[i]);
             }
-            o0.x = pack_bf16x2(v[0], v[1]);
-            o0.y = pack_bf16x2(v[2], v[3]);
-            o0.z = pack_bf16x2(v[4], v[5]);
-            o0.w = pack_bf16x2(v[6], v[7]);
-            *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out0) + off + 8 * q) = o0;
+            o0[q].x = pack_bf16x2(v[0], v[1]);
+            o0[q].y = pack_bf16x2(v[2], v[3]);
+            o0[q].z = pack_bf16x2(v[4], v[5]);
+            o0[q].w = pack_bf16x2(v[6], v[7]);
             if constexpr (EPI == EPI_GELU) {
-                uint4 o1;
-                o1.x = pack_bf16x2(gelu_f32(v[0]), gelu_f32(v[1]));
-                o1.y = pack_bf16x2(gelu_f32(v[2]), gelu_f32(v[3]));
-                o1.z = pack_bf16x2(gelu_f32(v[4]), gelu_f32(v[5]));
-                o1.w = pack_bf16x2(gelu_f32(v[6]), gelu_f32(v[7]));
-                *reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out1) + off + 8 * q) = o1;
+                o1[q].x = pack_bf16x2(gelu_fast(v[0]), gelu_fast(v[1]));
+                o1[q].y = pack_bf16x2(gelu_fast(v[2]), gelu_fast(v[3]));
+                o1[q].z = pack_bf16x2(gelu_fast(v[4]), gelu_fast(v[5]));
+                o1[q].w = pack_bf16x2(gelu_fast(v[6]), gelu_fast(v[7]));
             }
+        }
+        if (lane == 0) bulk_wait_read0();
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint32_t a = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
+            st_shared_v4(slot + a, o0[q]);
+            if constexpr (EPI == EPI_GELU) st_shared_v4(slot + 2048 + a, o1[q]);
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && any) {
+            tma_store_3d(tmO0, slot, col0, row0, 0);
+            if constexpr (EPI == EPI_GELU) tma_store_3d(tmO1, slot + 2048, col0, row0, 0);
+            bulk_commit();
         }
     }
 }
@@ -169,6 +233,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const uint32_t
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                    const GemmArgs g) {
     using C = TileCfg<BN>;
     constexpr int STAGES = C::STAGES;
@@ -179,7 +244,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * C::A_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+    uint8_t* sEpi = sB + STAGES * C::B_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiStagingBytes);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
     uint64_t* tfull = bars + 2 * STAGES;
@@ -355,7 +421,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        const int quad = warp & 3;  // tensor-memory lanes this warp may access
+        const int quad = warp & 3;              // tensor-memory lanes this warp may access
+        const int half = (warp - 2) / 4;        // which half of the tile's columns
+        constexpr int kChunks = BN / 64;        // 32-column chunks per half
+        const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
+        if (lane == 0) {
+            tma_prefetch_desc(&tmO0);
+            if (EPI == EPI_GELU) tma_prefetch_desc(&tmO1);
+        }
         int local = 0;
         for (int u = blockIdx.x; u < units; u += gridDim.x, ++local) {
             int mb, nb, split;
@@ -370,23 +443,26 @@ __global__ void __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int row = mb * kBM + quad * 32 + lane;
+            const int row0 = mb * kBM + quad * 32;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int i = 0; i < kChunks; ++i) {
+                const int c = half * kChunks + i;
                 uint32_t acc[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, acc);
                 tmem_wait_ld();
-                if (c == BN / 32 - 1) {
-                    // the whole accumulator is in registers: release it to the MMA warp
+                if (i == kChunks - 1) {
+                    // this warp's part of the accumulator is in registers: release it
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
                 }
-                epilogue_chunk<EPI>(g, acc, row, nb * BN + c * 32, split);
+                epilogue_chunk<EPI>(g, &tmO0, &tmO1, acc, row0, nb * BN + c * 32, split, slot, lane);
             }
         }
+        if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
+        __syncwarp();
     }
 
     tc_fence_before();

@@ -31,7 +31,7 @@ struct Tile2Cfg {
     static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
     static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
 constexpr int kPairM = 2 * kBM;  // 256 rows per pair tile
@@ -39,6 +39,7 @@ constexpr int kPairM = 2 * kBM;  // 256 rows per pair tile
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     const GemmArgs g) {
     using C = Tile2Cfg<BN>;
     constexpr int STAGES = C::STAGES;
@@ -49,7 +50,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                                                ~static_cast<uintptr_t>(1023));
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * C::A_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sB + STAGES * C::B_BYTES);
+    uint8_t* sEpi = sB + STAGES * C::B_BYTES;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiStagingBytes);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
     uint64_t* tfull = bars + 2 * STAGES;
@@ -227,7 +229,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
-        const int quad = warp & 3;
+        const int quad = warp & 3;            // tensor-memory lanes this warp may access
+        const int half = (warp - 2) / 4;      // which half of the tile's columns
+        constexpr int kChunks = BN / 64;      // 32-column chunks per half
+        const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
+        if (lane == 0) {
+            tma_prefetch_desc(&tmO0);
+            if (EPI == EPI_GELU) tma_prefetch_desc(&tmO1);
+        }
         int local = 0;
         for (int u = pair; u < units; u += npairs, ++local) {
             int mb, nb, split;
@@ -240,22 +249,25 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 break;
             }
             tc_fence_after();
-            const int row = mb * kPairM + static_cast<int>(rank) * kBM + quad * 32 + lane;
+            const int row0 = mb * kPairM + static_cast<int>(rank) * kBM + quad * 32;
             const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                    static_cast<uint32_t>(buf * BN);
 #pragma unroll 1
-            for (int c = 0; c < BN / 32; ++c) {
+            for (int i = 0; i < kChunks; ++i) {
+                const int c = half * kChunks + i;
                 uint32_t acc[32];
                 tmem_ld_32x32b_x32(t_row + c * 32, acc);
                 tmem_wait_ld();
-                if (c == BN / 32 - 1) {
+                if (i == kChunks - 1) {
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
                 }
-                epilogue_chunk<EPI>(g, acc, row, nb * BN + c * 32, split);
+                epilogue_chunk<EPI>(g, &tmO0, &tmO1, acc, row0, nb * BN + c * 32, split, slot, lane);
             }
         }
+        if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
+        __syncwarp();
     }
 
     tc_fence_before();

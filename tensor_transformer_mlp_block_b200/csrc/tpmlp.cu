@@ -101,6 +101,36 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int b
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Output of the epilogue's bulk stores: `planes` row-major M × N matrices
+// (one per K split) of bf16 or fp32, written in 32 × 32 boxes; bf16 boxes
+// are 64-byte rows with the 64-byte swizzle, fp32 boxes 128-byte rows with
+// the 128-byte swizzle (the layouts the epilogue stages in shared memory).
+// Box elements outside M × N are not written.
+bool make_out_map(CUtensorMap* m, void* ptr, int64_t planes, int64_t rows, int64_t cols, bool f32) {
+    EncodeTiledFn fn = encode_fn();
+    if (fn == nullptr) return false;
+    const cuuint64_t esize = f32 ? 4 : 2;
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
+                          static_cast<cuuint64_t>(planes)};
+    cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * esize,
+                             static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * esize};
+    cuuint32_t box[3] = {32u, 32u, 1u};
+    cuuint32_t estr[3] = {1u, 1u, 1u};
+    return fn(m, f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, ptr, dims,
+              strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              f32 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+bool make_out_maps(CUtensorMap* o0, CUtensorMap* o1, const GemmArgs& g, int M, int N, int splits) {
+    const bool f32 = (EPI == EPI_F32);
+    if (!make_out_map(o0, g.out0, f32 ? splits : 1, M, N, f32)) return false;
+    if (EPI == EPI_GELU) return make_out_map(o1, g.out1, 1, M, N, false);
+    *o1 = *o0;
+    return true;
+}
+
 tpmlp_status check_launch() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
     return cudaGetLastError() == cudaSuccess ? TPMLP_OK : TPMLP_ERR_CUDA;
@@ -175,7 +205,8 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     CUtensorMap tmA, tmB;
     const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
     const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN);
-    if (!okA || !okB) return TPMLP_ERR_CUDA;
+    CUtensorMap tmO0, tmO1;
+    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N, splits)) return TPMLP_ERR_CUDA;
     g.M = M;
     g.N = N;
     g.K = K;
@@ -200,7 +231,7 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     }
     const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
     const int grid = static_cast<int>(units < dev->num_sms ? units : dev->num_sms);
-    kern<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, g);
+    kern<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, tmO0, tmO1, g);
     return check_launch();
 }
 
@@ -214,7 +245,8 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     CUtensorMap tmA, tmB;
     const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
     const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN / 2);
-    if (!okA || !okB) return TPMLP_ERR_CUDA;
+    CUtensorMap tmO0, tmO1;
+    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N, splits)) return TPMLP_ERR_CUDA;
     g.M = M;
     g.N = N;
     g.K = K;
@@ -256,7 +288,7 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     }
     const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
     const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
-    kern<<<2 * pairs, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, g);
+    kern<<<2 * pairs, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, tmO0, tmO1, g);
     return check_launch();
 }
 
@@ -634,6 +666,19 @@ tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream) {
 }
 
 uint64_t tpmlp_launch_count(void) { return g_launches.load(); }
+
+tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t n, int form,
+                                   void* stream) {
+    cudaGetLastError();
+    if (n < 0 || (form != 0 && form != 1)) return TPMLP_ERR_INVALID;
+    if (n == 0) return TPMLP_OK;
+    if (!x || !y || !dy) return TPMLP_ERR_INVALID;
+    int64_t blocks = (n + 255) / 256;
+    if (blocks > 4096) blocks = 4096;
+    eval_activation_kernel<<<static_cast<unsigned>(blocks), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+        x, y, dy, n, form);
+    return check_launch();
+}
 
 void tpmlp_profile_enable(int on) { g_prof_on = (on != 0); }
 
