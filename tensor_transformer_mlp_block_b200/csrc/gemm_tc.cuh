@@ -69,7 +69,7 @@ struct TileCfg {
     static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
     // tensor-memory columns: two accumulators, rounded up to a power of two
     static constexpr int TMEM_COLS = (2 * BN <= 128) ? 128 : (2 * BN <= 256 ? 256 : 512);
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5 + 8) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
@@ -230,6 +230,126 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
     }
 }
 
+// The epilogue warps' loop over this CTA's work units (shared by the
+// one-CTA and the CTA-pair kernels). Each warp may read only the tensor-memory
+// lanes of its SM sub-partition (warp index mod 4), 32 accumulator rows.
+//
+// Plain epilogues (bias, fp32): all 8 warps drain their rows and store.
+// Epilogues with transcendental math (GeLU, GeLU′): the sub-partitions that
+// also host the TMA producer (warp 0) and the MMA issuer (warp 1) must stay
+// lightly loaded, or the math delays those latency-critical single threads
+// and the tensor pipe idles. There the 4 warps of sub-partitions 0 and 1 are
+// relays: they drain their rows from tensor memory and pass each raw fp32
+// 32 × 32 chunk through their shared-memory slot (128-byte swizzle,
+// conflict-free) to a partner warp in sub-partition 2 or 3, which computes
+// and stores both its own chunk and the relayed one. Hand-offs use one
+// full/empty mbarrier pair per relay (bounded waits).
+template <int BN, int EPI, bool PAIR>
+__device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
+                                              const CUtensorMap* tmO1, uint32_t tmem_base,
+                                              uint64_t* tfull, uint64_t* tempty, uint64_t* xfull,
+                                              uint64_t* xempty, uint8_t* sEpi, int u_first,
+                                              int u_stride, int units, int tile_rows,
+                                              int cta_row_off, volatile int* abort, uint64_t limit,
+                                              int warp, int lane) {
+    constexpr bool kRelay = (EPI == EPI_GELU || EPI == EPI_DGELU);
+    constexpr int kChunks = BN / 64;  // 32-column chunks per half of the tile
+    const int quad = warp & 3;          // tensor-memory lanes this warp may access
+    const int half = (warp - 2) / 4;    // which half of the tile's columns
+    const bool relay = kRelay && quad < 2;
+    const int pair_id = (quad & 1) + 2 * half;  // relay (quad 0/1) <-> math (quad 2/3)
+    const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
+    // a math warp's (quad 2/3) partner relay is warp 2 + 4·half + quad (quad - 2,
+    // same half), whose slot index is 4·half + quad
+    const uint32_t partner_slot = smem_u32(sEpi + (4 * half + quad) * kEpiSlotBytes);
+    if (lane == 0 && !relay) {
+        tma_prefetch_desc(tmO0);
+        if (EPI == EPI_GELU) tma_prefetch_desc(tmO1);
+    }
+    uint32_t xcount = 0;
+    int local = 0;
+    for (int u = u_first; u < units; u += u_stride, ++local) {
+        int mb, nb, split;
+        unit_coords(g, u, mb, nb, split);
+        const int buf = local & 1;
+        const uint32_t aphase = (local >> 1) & 1;
+        // every lane waits; the warp proceeds only if all lanes saw the
+        // phase complete, so the .sync.aligned loads below never diverge
+        const bool ok = mbar_wait_bounded(smem_u32(&tfull[buf]), aphase, abort, limit);
+        if (!__all_sync(0xffffffffu, ok)) {
+            raise_timeout(abort);
+            break;
+        }
+        tc_fence_after();
+        const int tile_row0 = mb * tile_rows + cta_row_off;
+        const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               static_cast<uint32_t>(buf * BN);
+        bool failed = false;
+#pragma unroll 1
+        for (int i = 0; i < kChunks; ++i) {
+            const int c = half * kChunks + i;
+            const int col0 = nb * BN + c * 32;
+            uint32_t acc[32];
+            tmem_ld_32x32b_x32(t_row + c * 32, acc);
+            tmem_wait_ld();
+            if (i == kChunks - 1) {
+                // this warp's part of the accumulator is in registers: release it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR)
+                        mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+                    else
+                        mbar_arrive(smem_u32(&tempty[buf]));
+                }
+            }
+            if (relay) {
+                const bool got = mbar_wait_bounded(smem_u32(&xempty[pair_id]), (xcount & 1u) ^ 1u,
+                                                   abort, limit);
+                if (!__all_sync(0xffffffffu, got)) {
+                    failed = true;
+                    break;
+                }
+#pragma unroll
+                for (int j = 0; j < 8; ++j)
+                    st_shared_v4(slot + lane * 128 + ((j ^ (lane & 7)) << 4),
+                                 make_uint4(acc[4 * j], acc[4 * j + 1], acc[4 * j + 2], acc[4 * j + 3]));
+                mbar_arrive(smem_u32(&xfull[pair_id]));
+                ++xcount;
+                continue;
+            }
+            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, split, slot, lane);
+            if constexpr (kRelay) {
+                // the partner relay's chunk: same columns, rows of quad - 2
+                const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
+                if (!__all_sync(0xffffffffu, got)) {
+                    failed = true;
+                    break;
+                }
+                uint32_t pacc[32];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const uint4 v = ld_shared_v4(partner_slot + lane * 128 + ((j ^ (lane & 7)) << 4));
+                    pacc[4 * j] = v.x;
+                    pacc[4 * j + 1] = v.y;
+                    pacc[4 * j + 2] = v.z;
+                    pacc[4 * j + 3] = v.w;
+                }
+                mbar_arrive(smem_u32(&xempty[pair_id]));
+                ++xcount;
+                epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, split,
+                                    slot, lane);
+            }
+        }
+        if (failed) {
+            raise_timeout(abort);
+            break;
+        }
+    }
+    if (lane == 0 && !relay) bulk_wait0();  // this warp's stores are complete before exit
+    __syncwarp();
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -251,13 +371,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t* tfull = bars + 2 * STAGES;
     uint64_t* tempty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    uint64_t* xfull = bars + 2 * STAGES + 5;   // relay hand-off, 4 pairs
+    uint64_t* xempty = bars + 2 * STAGES + 9;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 13);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
+        for (int x = 0; x < 4; ++x) {
+            mbar_init(smem_u32(&xfull[x]), 32);
+            mbar_init(smem_u32(&xempty[x]), 32);
+        }
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(smem_u32(&full[s]), 1);
             mbar_init(smem_u32(&empty[s]), 1);
@@ -421,48 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        const int quad = warp & 3;              // tensor-memory lanes this warp may access
-        const int half = (warp - 2) / 4;        // which half of the tile's columns
-        constexpr int kChunks = BN / 64;        // 32-column chunks per half
-        const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
-        if (lane == 0) {
-            tma_prefetch_desc(&tmO0);
-            if (EPI == EPI_GELU) tma_prefetch_desc(&tmO1);
-        }
-        int local = 0;
-        for (int u = blockIdx.x; u < units; u += gridDim.x, ++local) {
-            int mb, nb, split;
-            unit_coords(g, u, mb, nb, split);
-            const int buf = local & 1;
-            const uint32_t aphase = (local >> 1) & 1;
-            // every lane waits; the warp proceeds only if all lanes saw the
-            // phase complete, so the .sync.aligned loads below never diverge
-            const bool ok = mbar_wait_bounded(smem_u32(&tfull[buf]), aphase, abort, limit);
-            if (!__all_sync(0xffffffffu, ok)) {
-                raise_timeout(abort);
-                break;
-            }
-            tc_fence_after();
-            const int row0 = mb * kBM + quad * 32;
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                   static_cast<uint32_t>(buf * BN);
-#pragma unroll 1
-            for (int i = 0; i < kChunks; ++i) {
-                const int c = half * kChunks + i;
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(t_row + c * 32, acc);
-                tmem_wait_ld();
-                if (i == kChunks - 1) {
-                    // this warp's part of the accumulator is in registers: release it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(smem_u32(&tempty[buf]));
-                }
-                epilogue_chunk<EPI>(g, &tmO0, &tmO1, acc, row0, nb * BN + c * 32, split, slot, lane);
-            }
-        }
-        if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
-        __syncwarp();
+        epilogue_role<BN, EPI, false>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
+                                      blockIdx.x, gridDim.x, units, kBM, 0, abort, limit, warp, lane);
     }
 
     tc_fence_before();

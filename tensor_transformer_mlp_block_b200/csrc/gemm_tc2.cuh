@@ -30,7 +30,7 @@ struct Tile2Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
     static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
     static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5 + 8) + 16;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
@@ -57,7 +57,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t* tfull = bars + 2 * STAGES;
     uint64_t* tempty = bars + 2 * STAGES + 2;
     uint64_t* drain = bars + 2 * STAGES + 4;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 5);
+    uint64_t* xfull = bars + 2 * STAGES + 5;   // relay hand-off, 4 pairs
+    uint64_t* xempty = bars + 2 * STAGES + 9;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 13);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5;
@@ -77,6 +79,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&tempty[b]), 2 * kEpiWarps);
         }
         mbar_init(smem_u32(drain), 1);
+        for (int x = 0; x < 4; ++x) {
+            mbar_init(smem_u32(&xfull[x]), 32);
+            mbar_init(smem_u32(&xempty[x]), 32);
+        }
         *abort = 0;
         fence_mbar_init();
     }
@@ -229,45 +235,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
-        const int quad = warp & 3;            // tensor-memory lanes this warp may access
-        const int half = (warp - 2) / 4;      // which half of the tile's columns
-        constexpr int kChunks = BN / 64;      // 32-column chunks per half
-        const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
-        if (lane == 0) {
-            tma_prefetch_desc(&tmO0);
-            if (EPI == EPI_GELU) tma_prefetch_desc(&tmO1);
-        }
-        int local = 0;
-        for (int u = pair; u < units; u += npairs, ++local) {
-            int mb, nb, split;
-            unit_coords(g, u, mb, nb, split);
-            const int buf = local & 1;
-            const uint32_t aphase = (local >> 1) & 1;
-            const bool ok = mbar_wait_bounded(smem_u32(&tfull[buf]), aphase, abort, limit);
-            if (!__all_sync(0xffffffffu, ok)) {
-                raise_timeout(abort);
-                break;
-            }
-            tc_fence_after();
-            const int row0 = mb * kPairM + static_cast<int>(rank) * kBM + quad * 32;
-            const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
-                                   static_cast<uint32_t>(buf * BN);
-#pragma unroll 1
-            for (int i = 0; i < kChunks; ++i) {
-                const int c = half * kChunks + i;
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(t_row + c * 32, acc);
-                tmem_wait_ld();
-                if (i == kChunks - 1) {
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
-                }
-                epilogue_chunk<EPI>(g, &tmO0, &tmO1, acc, row0, nb * BN + c * 32, split, slot, lane);
-            }
-        }
-        if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
-        __syncwarp();
+        epilogue_role<BN, EPI, true>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
+                                     pair, npairs, units, kPairM, static_cast<int>(rank) * kBM, abort,
+                                     limit, warp, lane);
     }
 
     tc_fence_before();

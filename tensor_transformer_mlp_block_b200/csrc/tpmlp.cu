@@ -338,20 +338,42 @@ struct Plan {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
+// Shard groups S for the two row-parallel products (M = T, N = h, K = F).
+// S = 1 runs each output tile's K loop through all p shards in TMEM; S > 1
+// (a divisor of p, whole k-blocks per shard) gives each group of p/S shards
+// its own work units whose fp32 partials are then summed in order. The
+// automatic policy picks the S with the smallest estimated time:
+//   waves(S) · (k-blocks per unit + per-unit overhead) · t_kblock
+//   + the ordered reduction's bytes (S fp32 planes read, one bf16 written) / HBM rate,
+// with the tile geometry the launcher will use (256-row CTA-pair tiles when
+// T > 128, else 128-row tiles, 256 columns) and one unit per pair / SM in a wave.
 int choose_splits(int64_t T, int64_t h, int64_t F, int p, int num_sms) {
     const int64_t Fp = F / p;
     if (p == 1 || Fp % kBK != 0) return 1;
     const int policy = g_split_policy.load();
     if (policy == 1) return 1;
     if (policy == 2) return p;
-    const int64_t tiles = ((T + kBM - 1) / kBM) * ((h + 255) / 256);
-    int S = 1;
-    while (S < p && tiles * S < num_sms) {
-        int next = S + 1;
-        while (p % next != 0) ++next;
-        S = next;
+    const bool pairs = T > kBM;
+    const int64_t tile_m = pairs ? kPairM : kBM;
+    const int64_t tiles = ((T + tile_m - 1) / tile_m) * ((h + 255) / 256);
+    const int64_t slots = pairs ? num_sms / 2 : num_sms;
+    const double t_kb_us = pairs ? 0.284 : 0.142;  // one 64-deep k-block of a tile
+    const double overhead_kb = 8.0;                 // tile switch, epilogue tail
+    const int64_t k_blocks = (F + kBK - 1) / kBK;
+    int best = 1;
+    double best_us = 0.0;
+    for (int S = 1; S <= p; ++S) {
+        if (p % S != 0) continue;
+        const int64_t units = tiles * S;
+        const int64_t waves = (units + slots - 1) / slots;
+        double us = waves * (static_cast<double>(k_blocks) / S + overhead_kb) * t_kb_us;
+        if (S > 1) us += 3.0 + static_cast<double>(T) * h * (4.0 * S + 2.0) / 5.0e6;
+        if (S == 1 || us < best_us) {
+            best = S;
+            best_us = us;
+        }
     }
-    return S;
+    return best;
 }
 
 bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl) {
