@@ -47,6 +47,8 @@ def parse_args(argv=None):
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="7b")
     ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--graph", action="store_true",
+                    help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (for profiler runs)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -285,13 +287,32 @@ def bench_ours(args, cfg, world, rank, local):
         step()
     torch.cuda.synchronize()
     assert binding.last_device_status() == 0
+    n0 = binding.launch_count()
+    step()
+    torch.cuda.synchronize()
+    launches_per_step = binding.launch_count() - n0
+
+    run_step = step
+    if args.graph:
+        # one step captured once; replays re-launch the same kernels
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            step()
+        stream.wait_stream(side)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            step()
+        for _ in range(3):
+            graph.replay()
+        torch.cuda.synchronize()
+        run_step = graph.replay
 
     sampler = ClockSampler(physical_gpu_index(local))
     sampler.start()
     time.sleep(1.0)
     binding.profile_reset()
-    binding.profile_enable(True)
-    launches0 = binding.launch_count()
+    binding.profile_enable(not args.graph)
     barrier()
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -299,15 +320,24 @@ def bench_ours(args, cfg, world, rank, local):
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(args.steps):
-        step()
+        run_step()
     e1.record(stream)
     torch.cuda.synchronize()
     barrier()
     t_wall1 = time.time()
-    launches = binding.launch_count() - launches0
+    launches = launches_per_step * args.steps
     binding.profile_enable(False)
     kinds = binding.profile_collect()
     clocks = sampler.stop(t_wall0, t_wall1)
+    if args.graph:
+        # per-kernel times from a short eager pass (events cannot bracket graph replays)
+        binding.profile_reset()
+        binding.profile_enable(True)
+        for _ in range(min(args.steps, 20)):
+            step()
+        torch.cuda.synchronize()
+        binding.profile_enable(False)
+        kinds = binding.profile_collect()
     status = binding.last_device_status()
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -399,6 +429,7 @@ def bench_ours(args, cfg, world, rank, local):
         "data": "synthetic (seeded Gaussian inputs, random-init weights of the named shapes)",
         "config": {"workload": f"{cfg.name}-class TP-MLP fwd+bwd", "T": T, "h": h, "F": F, "p": p,
                    "flops_per_step": cfg.flops_fwd_bwd, "parallelism": f"replicas x{world}",
+                   "cuda_graph": bool(args.graph),
                    "l2": f"working set {working_set / 2**30:.2f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB "
                          "(inputs larger than L2; no flush)"},
         "frac_of_peak": {"measured_burst": agg["value"] / world / peaks["bf16_tflops"],

@@ -72,8 +72,40 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
     const int64_t r_end = min(R, r_begin + rows_per_chunk);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (VEC && c0 < C) {
-        // C % 8 == 0 and X 16-byte aligned: 8 columns are 16 (bf16) or 32 (fp32) bytes
-        for (int64_t r = r_begin + threadIdx.y; r < r_end; r += 8) {
+        // C % 8 == 0 and X 16-byte aligned: 8 columns are 16 (bf16) or 32 (fp32)
+        // bytes. Rows are visited in the same order as the scalar loop, but
+        // the loads of up to kU rows are issued before their additions so
+        // that many are in flight at once.
+        constexpr int kU = 8;
+        int64_t r = r_begin + threadIdx.y;
+        for (; r + 8 * (kU - 1) < r_end; r += 8 * kU) {
+            if constexpr (sizeof(T) == 2) {
+                uint4 raw[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u)
+                    raw[u] = __ldg(reinterpret_cast<const uint4*>(X + (r + 8 * u) * C + c0));
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    float f[8];
+                    unpack_bf16x8(raw[u], f);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) acc[i] += f[i];
+                }
+            } else {
+                float4 lo[kU], hi[kU];
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    lo[u] = __ldg(reinterpret_cast<const float4*>(X + (r + 8 * u) * C + c0));
+                    hi[u] = __ldg(reinterpret_cast<const float4*>(X + (r + 8 * u) * C + c0) + 1);
+                }
+#pragma unroll
+                for (int u = 0; u < kU; ++u) {
+                    acc[0] += lo[u].x; acc[1] += lo[u].y; acc[2] += lo[u].z; acc[3] += lo[u].w;
+                    acc[4] += hi[u].x; acc[5] += hi[u].y; acc[6] += hi[u].z; acc[7] += hi[u].w;
+                }
+            }
+        }
+        for (; r < r_end; r += 8) {
             const T* row = X + r * C + c0;
             if constexpr (sizeof(T) == 2) {
                 float f[8];
@@ -107,15 +139,39 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
     }
 }
 
-// Column sums, pass 2: out[c] = Σ_{chunk ascending} partial[chunk][c].
+// Column sums, pass 2: out[c] = Σ over chunks of partial[chunk][c]. Block
+// (32, 8): x picks one of 32 consecutive columns (coalesced reads), y one of 8
+// contiguous chunk groups; each thread adds its group's chunks in ascending
+// order, then the 8 group sums are added in ascending group order. Fixed
+// assignment and order: bit-reproducible.
 __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ partial,
                                                           int chunks, int64_t C,
                                                           float* __restrict__ out) {
-    const int64_t c = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-    if (c >= C) return;
+    __shared__ float grp[8][32];
+    const int64_t c = blockIdx.x * 32 + threadIdx.x;
+    const int per = (chunks + 7) / 8;
+    const int k0 = threadIdx.y * per;
+    const int k1 = min(chunks, k0 + per);
     float s = 0.0f;
-    for (int k = 0; k < chunks; ++k) s += partial[k * C + c];
-    out[c] = s;
+    if (c < C) {
+        int k = k0;
+        for (; k + 8 <= k1; k += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = partial[(k + u) * C + c];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) s += v[u];
+        }
+        for (; k < k1; ++k) s += partial[k * C + c];
+    }
+    grp[threadIdx.y][threadIdx.x] = s;
+    __syncthreads();
+    if (threadIdx.y == 0 && c < C) {
+        float t = grp[0][threadIdx.x];
+#pragma unroll
+        for (int y = 1; y < 8; ++y) t += grp[y][threadIdx.x];
+        out[c] = t;
+    }
 }
 
 // GeLU and GeLU′ of n values with either form the library uses:

@@ -235,16 +235,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
 // lanes of its SM sub-partition (warp index mod 4), 32 accumulator rows.
 //
 // The sub-partitions that also host the TMA producer (warp 0) and the MMA
-// issuer (warp 1) must stay lightly loaded: epilogue math and store traffic
+// issuer (warp 1) should stay lightly loaded: epilogue math and store traffic
 // there delay those latency-critical single threads and the tensor pipe
 // idles (measured: up to 0.1 ms per 7B GEMM for GeLU, 4–6% for fp32
-// outputs). So the 4 epilogue warps of sub-partitions 0 and 1 are relays:
-// they drain their rows from tensor memory and pass each raw fp32 32 × 32
-// chunk through their shared-memory slot (128-byte swizzle, conflict-free)
-// to a partner warp in sub-partition 2 or 3, which computes and stores both
-// its own chunk and the relayed one. Hand-offs use one full/empty mbarrier
-// pair per relay (bounded waits).
-template <int BN, int EPI, bool PAIR>
+// outputs). With RELAY, the 4 epilogue warps of sub-partitions 0 and 1
+// are relays: they drain their rows from tensor memory and pass each raw
+// fp32 32 × 32 chunk through their shared-memory slot (128-byte swizzle,
+// conflict-free) to a partner warp in sub-partition 2 or 3, which computes
+// and stores both its own chunk and the relayed one. Hand-offs use one
+// full/empty mbarrier pair per relay (bounded waits). Relaying doubles the
+// work of the computing warps, so it pays only when a tile's main loop is
+// long enough to hide it; the host picks the instantiation per launch.
+template <int BN, int EPI, bool PAIR, bool RELAY>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
                                               const CUtensorMap* tmO1, uint32_t tmem_base,
                                               uint64_t* tfull, uint64_t* tempty, uint64_t* xfull,
@@ -252,11 +254,10 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                                               int u_stride, int units, int tile_rows,
                                               int cta_row_off, volatile int* abort, uint64_t limit,
                                               int warp, int lane) {
-    constexpr bool kRelay = true;
     constexpr int kChunks = BN / 64;  // 32-column chunks per half of the tile
     const int quad = warp & 3;          // tensor-memory lanes this warp may access
     const int half = (warp - 2) / 4;    // which half of the tile's columns
-    const bool relay = kRelay && quad < 2;
+    const bool relay = RELAY && quad < 2;
     const int pair_id = (quad & 1) + 2 * half;  // relay (quad 0/1) <-> math (quad 2/3)
     const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
     // a math warp's (quad 2/3) partner relay is warp 2 + 4·half + quad (quad - 2,
@@ -303,7 +304,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                         mbar_arrive(smem_u32(&tempty[buf]));
                 }
             }
-            if (relay) {
+            if (RELAY && relay) {
                 const bool got = mbar_wait_bounded(smem_u32(&xempty[pair_id]), (xcount & 1u) ^ 1u,
                                                    abort, limit);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -319,7 +320,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 continue;
             }
             epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, split, slot, lane);
-            if constexpr (kRelay) {
+            if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
                 const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
                 if (!__all_sync(0xffffffffu, got)) {
@@ -350,7 +351,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     __syncwarp();
 }
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
@@ -547,7 +548,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps
-        epilogue_role<BN, EPI, false>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
+        epilogue_role<BN, EPI, false, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
                                       blockIdx.x, gridDim.x, units, kBM, 0, abort, limit, warp, lane);
     }
 

@@ -36,7 +36,7 @@ struct Tile2Cfg {
 
 constexpr int kPairM = 2 * kBM;  // 256 rows per pair tile
 
-template <int BN, bool A_MN, bool B_MN, int EPI>
+template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
@@ -235,7 +235,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
-        epilogue_role<BN, EPI, true>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
+        epilogue_role<BN, EPI, true, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
                                      pair, npairs, units, kPairM, static_cast<int>(rank) * kBM, abort,
                                      limit, warp, lane);
     }
