@@ -30,6 +30,8 @@ from .oracle import (  # noqa: F401
     forward_sharded,
     gelu,
     gelu_grad,
+    gelu_tanh,
+    gelu_tanh_grad,
     get_threads,
     normal_cdf,
     normal_pdf,

@@ -26,21 +26,33 @@ def _gelu_grad(x: float) -> float:
     return _phi_cdf(x) + x * math.exp(-0.5 * x * x) / math.sqrt(2.0 * math.pi)
 
 
-def mlp(X, A, a, B, b, dZ):
+def _gelu_tanh(x: float) -> float:
+    return 0.5 * x * (1.0 + math.tanh(math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)))
+
+
+def _gelu_tanh_grad(x: float) -> float:
+    u = math.sqrt(2.0 / math.pi) * (x + 0.044715 * x ** 3)
+    du = math.sqrt(2.0 / math.pi) * (1.0 + 3 * 0.044715 * x * x)
+    return 0.5 * (1.0 + math.tanh(u)) + 0.5 * x * (1.0 - math.tanh(u) ** 2) * du
+
+
+def mlp(X, A, a, B, b, dZ, act: int = 0):
     """X: T×h, A: h×F, a: F, B: F×h, b: h, dZ: T×h, as nested lists of floats.
+    act: 0 = exact GeLU, 1 = tanh approximation.
 
     Returns a dict of nested lists: H, Y, Z, dH, dX, dA, da, dB, db.
     """
+    g, dg = (_gelu_tanh, _gelu_tanh_grad) if act else (_gelu, _gelu_grad)
     T, h, F = len(X), len(X[0]), len(A[0])
     H = [[math.fsum([X[t][k] * A[k][f] for k in range(h)] + [a[f]]) for f in range(F)]
          for t in range(T)]
-    Y = [[_gelu(H[t][f]) for f in range(F)] for t in range(T)]
+    Y = [[g(H[t][f]) for f in range(F)] for t in range(T)]
     Z = [[math.fsum([Y[t][f] * B[f][j] for f in range(F)] + [b[j]]) for j in range(h)]
          for t in range(T)]
     db = [math.fsum(dZ[t][j] for t in range(T)) for j in range(h)]
     dB = [[math.fsum(Y[t][f] * dZ[t][j] for t in range(T)) for j in range(h)] for f in range(F)]
     dY = [[math.fsum(dZ[t][j] * B[f][j] for j in range(h)) for f in range(F)] for t in range(T)]
-    dH = [[dY[t][f] * _gelu_grad(H[t][f]) for f in range(F)] for t in range(T)]
+    dH = [[dY[t][f] * dg(H[t][f]) for f in range(F)] for t in range(T)]
     da = [math.fsum(dH[t][f] for t in range(T)) for f in range(F)]
     dA = [[math.fsum(X[t][k] * dH[t][f] for t in range(T)) for f in range(F)] for k in range(h)]
     dX = [[math.fsum(dH[t][f] * A[k][f] for f in range(F)) for k in range(h)] for t in range(T)]

@@ -47,19 +47,21 @@ def _bind(path: str):
     lib = ctypes.CDLL(path)
     lib.tpo_set_threads.argtypes = [ctypes.c_int]
     lib.tpo_get_threads.restype = ctypes.c_int
-    for name in ("tpo_normal_cdf", "tpo_normal_pdf", "tpo_gelu", "tpo_gelu_grad"):
+    for name in ("tpo_normal_cdf", "tpo_normal_pdf", "tpo_gelu", "tpo_gelu_grad", "tpo_gelu_tanh",
+                 "tpo_gelu_tanh_grad"):
         fn = getattr(lib, name)
         fn.argtypes = [ctypes.c_double]
         fn.restype = ctypes.c_double
     lib.tpo_colsum.argtypes = [_I64, _I64, _D, _D]
-    lib.tpo_forward.argtypes = [_I64, _I64, _I64] + [_D] * 8
-    lib.tpo_backward.argtypes = [_I64, _I64, _I64] + [_D] * 12
-    lib.tpo_forward_sharded.argtypes = [_I64, _I64, _I64, ctypes.c_int] + [_D] * 8
-    lib.tpo_forward_sharded.restype = ctypes.c_int
-    lib.tpo_backward_sharded.argtypes = [_I64, _I64, _I64, ctypes.c_int] + [_D] * 12
-    lib.tpo_backward_sharded.restype = ctypes.c_int
-    lib.tpo_rows.argtypes = [_I64, _I64, _I64] + [_D] * 6 + [_I64, _P64] + [_D] * 5
-    lib.tpo_cols.argtypes = [_I64, _I64, _I64] + [_D] * 5 + [_I64, _P64] + [_D] * 6
+    _c = ctypes.c_int
+    lib.tpo_forward_act.argtypes = [_I64, _I64, _I64] + [_D] * 8 + [_c]
+    lib.tpo_backward_act.argtypes = [_I64, _I64, _I64] + [_D] * 12 + [_c]
+    lib.tpo_forward_sharded_act.argtypes = [_I64, _I64, _I64, _c] + [_D] * 8 + [_c]
+    lib.tpo_forward_sharded_act.restype = _c
+    lib.tpo_backward_sharded_act.argtypes = [_I64, _I64, _I64, _c] + [_D] * 12 + [_c]
+    lib.tpo_backward_sharded_act.restype = _c
+    lib.tpo_rows_act.argtypes = [_I64, _I64, _I64] + [_D] * 6 + [_I64, _P64] + [_D] * 5 + [_c]
+    lib.tpo_cols_act.argtypes = [_I64, _I64, _I64] + [_D] * 5 + [_I64, _P64] + [_D] * 6 + [_c]
     return lib
 
 
@@ -96,6 +98,12 @@ class Oracle:
     def gelu_grad(self, x: float) -> float:
         return float(self._lib.tpo_gelu_grad(float(x)))
 
+    def gelu_tanh(self, x: float) -> float:
+        return float(self._lib.tpo_gelu_tanh(float(x)))
+
+    def gelu_tanh_grad(self, x: float) -> float:
+        return float(self._lib.tpo_gelu_tanh_grad(float(x)))
+
     def colsum(self, M) -> np.ndarray:
         M = _in(M)
         T, N = M.shape
@@ -103,14 +111,15 @@ class Oracle:
         self._lib.tpo_colsum(T, N, _ptr(M), _ptr(out))
         return out
 
-    def forward(self, X, A, a, B, b):
-        """Unsplit forward. Returns (H, Y, Z) in float64."""
+    def forward(self, X, A, a, B, b, act: int = 0):
+        """Unsplit forward. Returns (H, Y, Z) in float64. act: 0 = exact GeLU,
+        1 = tanh approximation."""
         X, A, a, B, b = map(_in, (X, A, a, B, b))
         T, h = X.shape
         F = A.shape[1]
         assert A.shape == (h, F) and a.shape == (F,) and B.shape == (F, h) and b.shape == (h,)
         H, Y, Z = np.empty((T, F)), np.empty((T, F)), np.empty((T, h))
-        self._lib.tpo_forward(T, h, F, *map(_ptr, (X, A, a, B, b, H, Y, Z)))
+        self._lib.tpo_forward_act(T, h, F, *map(_ptr, (X, A, a, B, b, H, Y, Z)), int(act))
         return H, Y, Z
 
     @staticmethod
@@ -118,41 +127,43 @@ class Oracle:
         return dict(dH=np.empty((T, F)), dX=np.empty((T, h)), dA=np.empty((h, F)),
                     da=np.empty(F), dB=np.empty((F, h)), db=np.empty(h))
 
-    def backward(self, X, A, B, H, Y, dZ):
+    def backward(self, X, A, B, H, Y, dZ, act: int = 0):
         """Unsplit backward. Returns dict with dH, dX, dA, da, dB, db (float64)."""
         X, A, B, H, Y, dZ = map(_in, (X, A, B, H, Y, dZ))
         T, h = X.shape
         F = A.shape[1]
         out = self._grads(T, h, F)
-        self._lib.tpo_backward(T, h, F, *map(_ptr, (X, A, B, H, Y, dZ)),
-                               *map(_ptr, (out[k] for k in ("dH", "dX", "dA", "da", "dB", "db"))))
+        self._lib.tpo_backward_act(T, h, F, *map(_ptr, (X, A, B, H, Y, dZ)),
+                                   *map(_ptr, (out[k] for k in ("dH", "dX", "dA", "da", "dB", "db"))),
+                                   int(act))
         return out
 
-    def forward_sharded(self, X, A, a, B, b, p: int):
+    def forward_sharded(self, X, A, a, B, b, p: int, act: int = 0):
         """Forward through the p-way column/row partition. Returns (H, Y, Z)."""
         X, A, a, B, b = map(_in, (X, A, a, B, b))
         T, h = X.shape
         F = A.shape[1]
         H, Y, Z = np.empty((T, F)), np.empty((T, F)), np.empty((T, h))
-        rc = self._lib.tpo_forward_sharded(T, h, F, int(p), *map(_ptr, (X, A, a, B, b, H, Y, Z)))
+        rc = self._lib.tpo_forward_sharded_act(T, h, F, int(p), *map(_ptr, (X, A, a, B, b, H, Y, Z)),
+                                               int(act))
         if rc != 0:
             raise ValueError(f"p={p} does not divide F={F}")
         return H, Y, Z
 
-    def backward_sharded(self, X, A, B, H, Y, dZ, p: int):
+    def backward_sharded(self, X, A, B, H, Y, dZ, p: int, act: int = 0):
         """Backward through the p-way partition (dX summed over shards in order)."""
         X, A, B, H, Y, dZ = map(_in, (X, A, B, H, Y, dZ))
         T, h = X.shape
         F = A.shape[1]
         out = self._grads(T, h, F)
-        rc = self._lib.tpo_backward_sharded(
+        rc = self._lib.tpo_backward_sharded_act(
             T, h, F, int(p), *map(_ptr, (X, A, B, H, Y, dZ)),
-            *map(_ptr, (out[k] for k in ("dH", "dX", "dA", "da", "dB", "db"))))
+            *map(_ptr, (out[k] for k in ("dH", "dX", "dA", "da", "dB", "db"))), int(act))
         if rc != 0:
             raise ValueError(f"p={p} does not divide F={F}")
         return out
 
-    def rows(self, X, A, a, B, b, dZ, R):
+    def rows(self, X, A, a, B, b, dZ, R, act: int = 0):
         """Outputs restricted to token rows R: dict with H, Y, Z, dH, dX."""
         X, A, a, B, b, dZ = map(_in, (X, A, a, B, b, dZ))
         R = np.ascontiguousarray(np.asarray(R, dtype=np.int64))
@@ -162,11 +173,11 @@ class Oracle:
         n = len(R)
         out = dict(H=np.empty((n, F)), Y=np.empty((n, F)), Z=np.empty((n, h)),
                    dH=np.empty((n, F)), dX=np.empty((n, h)))
-        self._lib.tpo_rows(T, h, F, *map(_ptr, (X, A, a, B, b, dZ)), n, R.ctypes.data_as(_P64),
-                           *map(_ptr, (out[k] for k in ("H", "Y", "Z", "dH", "dX"))))
+        self._lib.tpo_rows_act(T, h, F, *map(_ptr, (X, A, a, B, b, dZ)), n, R.ctypes.data_as(_P64),
+                               *map(_ptr, (out[k] for k in ("H", "Y", "Z", "dH", "dX"))), int(act))
         return out
 
-    def cols(self, X, A, a, B, dZ, J):
+    def cols(self, X, A, a, B, dZ, J, act: int = 0):
         """Outputs restricted to hidden columns J: dict with H, Y, dH (T × |J|),
         dA (h × |J|), da (|J|), dB (|J| × h)."""
         X, A, a, B, dZ = map(_in, (X, A, a, B, dZ))
@@ -177,8 +188,9 @@ class Oracle:
         n = len(J)
         out = dict(H=np.empty((T, n)), Y=np.empty((T, n)), dH=np.empty((T, n)),
                    dA=np.empty((h, n)), da=np.empty(n), dB=np.empty((n, h)))
-        self._lib.tpo_cols(T, h, F, *map(_ptr, (X, A, a, B, dZ)), n, J.ctypes.data_as(_P64),
-                           *map(_ptr, (out[k] for k in ("H", "Y", "dH", "dA", "da", "dB"))))
+        self._lib.tpo_cols_act(T, h, F, *map(_ptr, (X, A, a, B, dZ)), n, J.ctypes.data_as(_P64),
+                               *map(_ptr, (out[k] for k in ("H", "Y", "dH", "dA", "da", "dB"))),
+                               int(act))
         return out
 
 
@@ -234,25 +246,33 @@ def colsum(M):
     return default().colsum(M)
 
 
-def forward(X, A, a, B, b):
-    return default().forward(X, A, a, B, b)
+def gelu_tanh(x):
+    return default().gelu_tanh(x)
 
 
-def backward(X, A, B, H, Y, dZ):
-    return default().backward(X, A, B, H, Y, dZ)
+def gelu_tanh_grad(x):
+    return default().gelu_tanh_grad(x)
 
 
-def forward_sharded(X, A, a, B, b, p):
-    return default().forward_sharded(X, A, a, B, b, p)
+def forward(X, A, a, B, b, act=0):
+    return default().forward(X, A, a, B, b, act)
 
 
-def backward_sharded(X, A, B, H, Y, dZ, p):
-    return default().backward_sharded(X, A, B, H, Y, dZ, p)
+def backward(X, A, B, H, Y, dZ, act=0):
+    return default().backward(X, A, B, H, Y, dZ, act)
 
 
-def rows(X, A, a, B, b, dZ, R):
-    return default().rows(X, A, a, B, b, dZ, R)
+def forward_sharded(X, A, a, B, b, p, act=0):
+    return default().forward_sharded(X, A, a, B, b, p, act)
 
 
-def cols(X, A, a, B, dZ, J):
-    return default().cols(X, A, a, B, dZ, J)
+def backward_sharded(X, A, B, H, Y, dZ, p, act=0):
+    return default().backward_sharded(X, A, B, H, Y, dZ, p, act)
+
+
+def rows(X, A, a, B, b, dZ, R, act=0):
+    return default().rows(X, A, a, B, b, dZ, R, act)
+
+
+def cols(X, A, a, B, dZ, J, act=0):
+    return default().cols(X, A, a, B, dZ, J, act)

@@ -36,6 +36,10 @@
  * The tpo_*_sharded functions follow the pages' partition literally
  * (per-shard products concatenated or summed over i = 1..p) and exist so the
  * tests can check the pages' two identities against the unsplit functions.
+ *
+ * Each path function has an _act form whose last argument selects the
+ * activation: 0 = the exact GeLU above, 1 = the tanh approximation
+ * (tpo_gelu_tanh). The form without the suffix is act = 0.
  */
 #include <math.h>
 #include <stdint.h>
@@ -75,6 +79,32 @@ double tpo_gelu(double x) { return x * tpo_normal_cdf(x); }
 
 /* d/dx [x·Φ(x)] = Φ(x) + x·φ(x). */
 double tpo_gelu_grad(double x) { return tpo_normal_cdf(x) + x * tpo_normal_pdf(x); }
+
+/* The tanh approximation of GeLU (Hendrycks & Gimpel, "Gaussian Error Linear
+ * Units", 2016): ½·x·(1 + tanh(u)), u = √(2/π)·(x + 0.044715·x³). Offered as
+ * a variant; the exact form above is the reading of the pages' "gelu". */
+#define TPO_SQRT_2_OVER_PI 0.79788456080286535588 /* √(2/π) */
+#define TPO_GELU_TANH_C 0.044715
+
+double tpo_gelu_tanh(double x) {
+    const double u = TPO_SQRT_2_OVER_PI * (x + TPO_GELU_TANH_C * x * x * x);
+    return 0.5 * x * (1.0 + tanh(u));
+}
+
+/* d/dx of the tanh form: ½(1 + tanh u) + ½·x·(1 − tanh² u)·du/dx,
+ * du/dx = √(2/π)·(1 + 3·0.044715·x²). */
+double tpo_gelu_tanh_grad(double x) {
+    const double u = TPO_SQRT_2_OVER_PI * (x + TPO_GELU_TANH_C * x * x * x);
+    const double th = tanh(u);
+    const double du = TPO_SQRT_2_OVER_PI * (1.0 + 3.0 * TPO_GELU_TANH_C * x * x);
+    return 0.5 * (1.0 + th) + 0.5 * x * (1.0 - th * th) * du;
+}
+
+/* Activation selector: 0 = exact GeLU, 1 = tanh approximation. */
+static double tpo_act(int act, double x) { return act ? tpo_gelu_tanh(x) : tpo_gelu(x); }
+static double tpo_act_grad(int act, double x) {
+    return act ? tpo_gelu_tanh_grad(x) : tpo_gelu_grad(x);
+}
 
 /* C[m, n] (+)= Σ_k P[m, k]·Q[k, n] for P (M × K), Q (K × N), row-major.
  * The k loop is the middle loop so each C row is updated with Q's rows in
@@ -136,15 +166,15 @@ void tpo_colsum(int64_t T, int64_t N, const double* Mat, double* out) {
 }
 
 /* Forward of the unsplit block. */
-void tpo_forward(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+void tpo_forward_act(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
                  const double* a, const double* B, const double* b, double* H, double* Y,
-                 double* Z) {
+                 double* Z, int act) {
     mm_nn(T, F, h, X, A, H, 0);
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t)
         for (int64_t f = 0; f < F; ++f) {
             H[t * F + f] += a[f];
-            Y[t * F + f] = tpo_gelu(H[t * F + f]);
+            Y[t * F + f] = tpo_act(act, H[t * F + f]);
         }
     mm_nn(T, h, F, Y, B, Z, 0);
 #pragma omp parallel for schedule(static)
@@ -152,20 +182,33 @@ void tpo_forward(int64_t T, int64_t h, int64_t F, const double* X, const double*
         for (int64_t j = 0; j < h; ++j) Z[t * h + j] += b[j];
 }
 
+void tpo_forward(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+                 const double* a, const double* B, const double* b, double* H, double* Y,
+                 double* Z) {
+    tpo_forward_act(T, h, F, X, A, a, B, b, H, Y, Z, 0);
+}
+
 /* Backward of the unsplit block, given the forward's H and Y. */
-void tpo_backward(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+void tpo_backward_act(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
                   const double* B, const double* H, const double* Y, const double* dZ,
                   double* dH, double* dX, double* dA, double* da, double* dB,
-                  double* db) {
+                  double* db, int act) {
     tpo_colsum(T, h, dZ, db);
     mm_tn(F, h, T, Y, dZ, dB);
     mm_nt(T, F, h, dZ, B, dH); /* dH holds dY = dZ·Bᵀ here */
 #pragma omp parallel for schedule(static)
     for (int64_t t = 0; t < T; ++t)
-        for (int64_t f = 0; f < F; ++f) dH[t * F + f] *= tpo_gelu_grad(H[t * F + f]);
+        for (int64_t f = 0; f < F; ++f) dH[t * F + f] *= tpo_act_grad(act, H[t * F + f]);
     tpo_colsum(T, F, dH, da);
     mm_tn(h, F, T, X, dH, dA);
     mm_nt(T, h, F, dH, A, dX);
+}
+
+void tpo_backward(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+                  const double* B, const double* H, const double* Y, const double* dZ,
+                  double* dH, double* dX, double* dA, double* da, double* dB,
+                  double* db) {
+    tpo_backward_act(T, h, F, X, A, B, H, Y, dZ, dH, dX, dA, da, dB, db, 0);
 }
 
 /* Copy the column block [c0, c0 + nc) of a row-major R × C matrix. */
@@ -181,9 +224,9 @@ static double* col_block(int64_t R, int64_t C, const double* M, int64_t c0, int6
  * partial products P_i = Y_i·B_i are formed separately and summed over
  * i = 1..p in order (the all-reduce), then b is added once. Returns 0, or -1
  * if p does not divide F. */
-int tpo_forward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
+int tpo_forward_sharded_act(int64_t T, int64_t h, int64_t F, int p, const double* X,
                         const double* A, const double* a, const double* B, const double* b,
-                        double* H, double* Y, double* Z) {
+                        double* H, double* Y, double* Z, int act) {
     if (p < 1 || F % p != 0) return -1;
     const int64_t Fp = F / p;
     double* Hi = (double*)malloc((size_t)(T * Fp) * sizeof(double));
@@ -197,7 +240,7 @@ int tpo_forward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
             for (int64_t f = 0; f < Fp; ++f) {
                 double v = Hi[t * Fp + f] + a[i * Fp + f];
                 H[t * F + i * Fp + f] = v;
-                Yi[t * Fp + f] = tpo_gelu(v);
+                Yi[t * Fp + f] = tpo_act(act, v);
                 Y[t * F + i * Fp + f] = Yi[t * Fp + f];
             }
         mm_nn(T, h, Fp, Yi, B + (int64_t)i * Fp * h, Pi, 0);
@@ -212,14 +255,20 @@ int tpo_forward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
     return 0;
 }
 
+int tpo_forward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
+                        const double* A, const double* a, const double* B, const double* b,
+                        double* H, double* Y, double* Z) {
+    return tpo_forward_sharded_act(T, h, F, p, X, A, a, B, b, H, Y, Z, 0);
+}
+
 /* Backward through the partition. Per shard, with no exchange:
  * dY_i = dZ·B_iᵀ, dH_i = dY_i ⊙ GeLU′(H_i), dA_i = Xᵀ·dH_i, da_i = 1ᵀ·dH_i,
  * dB_i = Y_iᵀ·dZ. X is replicated, so its gradient is the sum over shards of
  * dH_i·A_iᵀ, taken in order i = 1..p. db = 1ᵀ·dZ. */
-int tpo_backward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
+int tpo_backward_sharded_act(int64_t T, int64_t h, int64_t F, int p, const double* X,
                          const double* A, const double* B, const double* H, const double* Y,
                          const double* dZ, double* dH, double* dX, double* dA, double* da,
-                         double* dB, double* db) {
+                         double* dB, double* db, int act) {
     if (p < 1 || F % p != 0) return -1;
     const int64_t Fp = F / p;
     double* Pi = (double*)malloc((size_t)(T * h) * sizeof(double));
@@ -233,7 +282,7 @@ int tpo_backward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X
         double* dHi = (double*)malloc((size_t)(T * Fp) * sizeof(double));
         double* dAi = (double*)malloc((size_t)(h * Fp) * sizeof(double));
         mm_nt(T, Fp, h, dZ, Bi, dHi);
-        for (int64_t e = 0; e < T * Fp; ++e) dHi[e] *= tpo_gelu_grad(Hi[e]);
+        for (int64_t e = 0; e < T * Fp; ++e) dHi[e] *= tpo_act_grad(act, Hi[e]);
         mm_tn(h, Fp, T, X, dHi, dAi);
         mm_tn(Fp, h, T, Yi, dZ, dB + (int64_t)i * Fp * h);
         tpo_colsum(T, Fp, dHi, da + i * Fp);
@@ -253,14 +302,21 @@ int tpo_backward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X
     return 0;
 }
 
+int tpo_backward_sharded(int64_t T, int64_t h, int64_t F, int p, const double* X,
+                         const double* A, const double* B, const double* H, const double* Y,
+                         const double* dZ, double* dH, double* dX, double* dA, double* da,
+                         double* dB, double* db) {
+    return tpo_backward_sharded_act(T, h, F, p, X, A, B, H, Y, dZ, dH, dX, dA, da, dB, db, 0);
+}
+
 /* The forward and backward restricted to the token rows R (nR of them).
  * Outputs are nR-row matrices: H_R, Y_R, dH_R (nR × F) and Z_R, dX_R (nR × h).
  * Each needs only its own rows: H[r, :] = X[r, :]·A + a, Z[r, :] = Y[r, :]·B + b,
  * dH[r, :] = (dZ[r, :]·Bᵀ) ⊙ GeLU′(H[r, :]), dX[r, :] = dH[r, :]·Aᵀ. */
-void tpo_rows(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+void tpo_rows_act(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
               const double* a, const double* B, const double* b, const double* dZ,
               int64_t nR, const int64_t* R, double* H_R, double* Y_R, double* Z_R,
-              double* dH_R, double* dX_R) {
+              double* dH_R, double* dX_R, int act) {
     (void)T;
     double* XR = (double*)malloc((size_t)(nR * h) * sizeof(double));
     double* dZR = (double*)malloc((size_t)(nR * h) * sizeof(double));
@@ -272,16 +328,23 @@ void tpo_rows(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
     for (int64_t r = 0; r < nR; ++r)
         for (int64_t f = 0; f < F; ++f) {
             H_R[r * F + f] += a[f];
-            Y_R[r * F + f] = tpo_gelu(H_R[r * F + f]);
+            Y_R[r * F + f] = tpo_act(act, H_R[r * F + f]);
         }
     mm_nn(nR, h, F, Y_R, B, Z_R, 0);
     for (int64_t r = 0; r < nR; ++r)
         for (int64_t j = 0; j < h; ++j) Z_R[r * h + j] += b[j];
     mm_nt(nR, F, h, dZR, B, dH_R);
-    for (int64_t e = 0; e < nR * F; ++e) dH_R[e] *= tpo_gelu_grad(H_R[e]);
+    for (int64_t e = 0; e < nR * F; ++e) dH_R[e] *= tpo_act_grad(act, H_R[e]);
     mm_nt(nR, h, F, dH_R, A, dX_R);
     free(XR);
     free(dZR);
+}
+
+void tpo_rows(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+              const double* a, const double* B, const double* b, const double* dZ,
+              int64_t nR, const int64_t* R, double* H_R, double* Y_R, double* Z_R,
+              double* dH_R, double* dX_R) {
+    tpo_rows_act(T, h, F, X, A, a, B, b, dZ, nR, R, H_R, Y_R, Z_R, dH_R, dX_R, 0);
 }
 
 /* The forward and backward restricted to the hidden columns J of F (nJ of
@@ -290,10 +353,10 @@ void tpo_rows(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
  * H[:, f] = X·A[:, f] + a[f], dY[:, f] = dZ·B[f, :]ᵀ, dH[:, f] = dY[:, f] ⊙
  * GeLU′(H[:, f]), dA[:, f] = Xᵀ·dH[:, f], da[f] = 1ᵀ·dH[:, f],
  * dB[f, :] = Y[:, f]ᵀ·dZ. */
-void tpo_cols(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+void tpo_cols_act(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
               const double* a, const double* B, const double* dZ, int64_t nJ,
               const int64_t* J, double* H_J, double* Y_J, double* dH_J, double* dA_J,
-              double* da_J, double* dB_J) {
+              double* da_J, double* dB_J, int act) {
     double* AJ = (double*)malloc((size_t)(h * nJ) * sizeof(double)); /* h × nJ */
     double* BJ = (double*)malloc((size_t)(nJ * h) * sizeof(double)); /* nJ × h */
     for (int64_t k = 0; k < h; ++k)
@@ -303,13 +366,20 @@ void tpo_cols(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
     for (int64_t t = 0; t < T; ++t)
         for (int64_t c = 0; c < nJ; ++c) {
             H_J[t * nJ + c] += a[J[c]];
-            Y_J[t * nJ + c] = tpo_gelu(H_J[t * nJ + c]);
+            Y_J[t * nJ + c] = tpo_act(act, H_J[t * nJ + c]);
         }
     mm_nt(T, nJ, h, dZ, BJ, dH_J);
-    for (int64_t e = 0; e < T * nJ; ++e) dH_J[e] *= tpo_gelu_grad(H_J[e]);
+    for (int64_t e = 0; e < T * nJ; ++e) dH_J[e] *= tpo_act_grad(act, H_J[e]);
     mm_tn(h, nJ, T, X, dH_J, dA_J);
     tpo_colsum(T, nJ, dH_J, da_J);
     mm_tn(nJ, h, T, Y_J, dZ, dB_J);
     free(AJ);
     free(BJ);
+}
+
+void tpo_cols(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
+              const double* a, const double* B, const double* dZ, int64_t nJ,
+              const int64_t* J, double* H_J, double* Y_J, double* dH_J, double* dA_J,
+              double* da_J, double* dB_J) {
+    tpo_cols_act(T, h, F, X, A, a, B, dZ, nJ, J, H_J, Y_J, dH_J, dA_J, da_J, dB_J, 0);
 }

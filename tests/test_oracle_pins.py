@@ -39,9 +39,9 @@ def _rand_problem(rng, T, h, F, scale_w=0.7, scale_b=0.5):
                 b=rng.standard_normal(h) * scale_b, dZ=rng.standard_normal((T, h)))
 
 
-def _all_outputs(orc, P):
-    H, Y, Z = orc.forward(P["X"], P["A"], P["a"], P["B"], P["b"])
-    g = orc.backward(P["X"], P["A"], P["B"], H, Y, P["dZ"])
+def _all_outputs(orc, P, act=0):
+    H, Y, Z = orc.forward(P["X"], P["A"], P["a"], P["B"], P["b"], act)
+    g = orc.backward(P["X"], P["A"], P["B"], H, Y, P["dZ"], act)
     return dict(H=H, Y=Y, Z=Z, **g)
 
 
@@ -89,6 +89,26 @@ def check_gelu_grad_fd(orc):
 
 def test_gelu_grad_matches_finite_difference():
     check_gelu_grad_fd(oracle.default())
+
+
+def test_gelu_tanh_closed_forms():
+    """The tanh form ½x(1 + tanh(√(2/π)(x + 0.044715x³))): value and slope at
+    0, the identity g(x) − g(−x) = x (tanh is odd), the tails, its derivative
+    against a central difference, and its distance from the exact GeLU (which
+    the normal table pins) staying below 5e-4 everywhere."""
+    o = oracle.default()
+    assert o.gelu_tanh(0.0) == 0.0 and o.gelu_tanh_grad(0.0) == 0.5
+    assert o.gelu_tanh(10.0) == 10.0 and abs(o.gelu_tanh(-10.0)) < 1e-20
+    xs = np.linspace(-6, 6, 241)
+    for x in xs:
+        assert abs(o.gelu_tanh(x) - o.gelu_tanh(-x) - x) < 1e-14
+        fd = (o.gelu_tanh(x + 1e-5) - o.gelu_tanh(x - 1e-5)) / 2e-5
+        assert abs(fd - o.gelu_tanh_grad(x)) < 1e-9, x
+    worst = max(abs(o.gelu_tanh(x) - o.gelu(x)) for x in np.linspace(-8, 8, 3201))
+    assert 1e-4 < worst < 5e-4
+    # at x = 1: u = √(2/π)·1.044715, from the textbook value of √(2/π)
+    u = 0.7978845608028654 * 1.044715
+    assert abs(o.gelu_tanh(1.0) - 0.5 * (1 + math.tanh(u))) < 1e-15
 
 
 # --------------------------------------------------------- hand-worked example
@@ -143,33 +163,34 @@ def test_hand_worked_example():
 BRUTE_SHAPES = [(1, 1, 1), (2, 3, 4), (3, 2, 8), (5, 4, 12), (8, 6, 24), (7, 5, 10)]
 
 
-def check_bruteforce(orc, shapes=BRUTE_SHAPES, seed=0):
+def check_bruteforce(orc, shapes=BRUTE_SHAPES, seed=0, act=0):
     rng = np.random.default_rng(seed)
     for T, h, F in shapes:
         P = _rand_problem(rng, T, h, F)
-        got = _all_outputs(orc, P)
-        ref = bruteforce.mlp(*(P[k].tolist() for k in ("X", "A", "a", "B", "b", "dZ")))
+        got = _all_outputs(orc, P, act)
+        ref = bruteforce.mlp(*(P[k].tolist() for k in ("X", "A", "a", "B", "b", "dZ")), act=act)
         for k, v in ref.items():
-            assert _max_rel(got[k], v) <= 1e-12, (k, T, h, F)
+            assert _max_rel(got[k], v) <= 1e-12, (k, T, h, F, act)
 
 
-def test_bruteforce_tiny():
-    check_bruteforce(oracle.default())
+@pytest.mark.parametrize("act", [0, 1])
+def test_bruteforce_tiny(act):
+    check_bruteforce(oracle.default(), act=act)
 
 
 # -------------------------------------------------------- finite differences
 
-def check_finite_differences(orc, seed=1, T=5, h=4, F=8, n_probe=6):
+def check_finite_differences(orc, seed=1, T=5, h=4, F=8, n_probe=6, act=0):
     """L = Σ dZ ⊙ Z is linear in Z, so ∂L/∂θ is exactly the backward's output
     for θ ∈ {X, A, a, B, b}. Central differences (ε = 1e-6) pin all five
     gradients, GeLU′ included, independently of the backward formulas."""
     rng = np.random.default_rng(seed)
     P = _rand_problem(rng, T, h, F)
-    out = _all_outputs(orc, P)
+    out = _all_outputs(orc, P, act)
     grad_of = {"X": out["dX"], "A": out["dA"], "a": out["da"], "B": out["dB"], "b": out["db"]}
 
     def loss(Q):
-        _, _, Z = orc.forward(Q["X"], Q["A"], Q["a"], Q["B"], Q["b"])
+        _, _, Z = orc.forward(Q["X"], Q["A"], Q["a"], Q["B"], Q["b"], act)
         return float(np.sum(P["dZ"] * Z))
 
     eps = 1e-6
@@ -185,33 +206,35 @@ def check_finite_differences(orc, seed=1, T=5, h=4, F=8, n_probe=6):
             assert abs(fd - an) <= 1e-7 * max(1.0, abs(an)), (name, idx, fd, an)
 
 
-def test_finite_differences():
-    check_finite_differences(oracle.default())
+@pytest.mark.parametrize("act", [0, 1])
+def test_finite_differences(act):
+    check_finite_differences(oracle.default(), act=act)
 
 
 # -------------------------------------------------- the pages' two identities
 
-def check_partition_identities(orc, seed=2, T=6, h=5, F=24):
+def check_partition_identities(orc, seed=2, T=6, h=5, F=24, act=0):
     rng = np.random.default_rng(seed)
     P = _rand_problem(rng, T, h, F)
-    H, Y, Z = orc.forward(P["X"], P["A"], P["a"], P["B"], P["b"])
-    g = orc.backward(P["X"], P["A"], P["B"], H, Y, P["dZ"])
+    H, Y, Z = orc.forward(P["X"], P["A"], P["a"], P["B"], P["b"], act)
+    g = orc.backward(P["X"], P["A"], P["B"], H, Y, P["dZ"], act)
     for p in [d for d in range(1, F + 1) if F % d == 0]:
-        Hs, Ys, Zs = orc.forward_sharded(P["X"], P["A"], P["a"], P["B"], P["b"], p)
+        Hs, Ys, Zs = orc.forward_sharded(P["X"], P["A"], P["a"], P["B"], P["b"], p, act)
         # column split: concatenation of X·A_i + a_i is X·A + a, column for column
         np.testing.assert_array_equal(Hs, H)
         np.testing.assert_array_equal(Ys, Y)
         # row split: Σ_i Y_i·B_i equals Y·B (rounding order differs)
         assert _max_rel(Zs, Z) < 1e-13, p
-        gs = orc.backward_sharded(P["X"], P["A"], P["B"], Hs, Ys, P["dZ"], p)
+        gs = orc.backward_sharded(P["X"], P["A"], P["B"], Hs, Ys, P["dZ"], p, act)
         for k in g:
             assert _max_rel(gs[k], g[k]) < 1e-13, (k, p)
     with pytest.raises(ValueError):
         orc.forward_sharded(P["X"], P["A"], P["a"], P["B"], P["b"], 5)
 
 
-def test_partition_identities():
-    check_partition_identities(oracle.default())
+@pytest.mark.parametrize("act", [0, 1])
+def test_partition_identities(act):
+    check_partition_identities(oracle.default(), act=act)
 
 
 def test_shard_split_by_hand():
@@ -286,17 +309,18 @@ def test_empty_tokens():
 
 # --------------------------------------------------------- subset functions
 
-def test_rows_and_cols_match_full():
+@pytest.mark.parametrize("act", [0, 1])
+def test_rows_and_cols_match_full(act):
     rng = np.random.default_rng(6)
     T, h, F = 9, 5, 12
     P = _rand_problem(rng, T, h, F)
-    full = _all_outputs(oracle.default(), P)
+    full = _all_outputs(oracle.default(), P, act)
     R = [0, 3, 8]
-    r = oracle.rows(P["X"], P["A"], P["a"], P["B"], P["b"], P["dZ"], R)
+    r = oracle.rows(P["X"], P["A"], P["a"], P["B"], P["b"], P["dZ"], R, act)
     for k in ("H", "Y", "Z", "dH", "dX"):
         np.testing.assert_allclose(r[k], full[k][R], rtol=1e-14, atol=1e-15, err_msg=k)
     J = [1, 4, 11]
-    c = oracle.cols(P["X"], P["A"], P["a"], P["B"], P["dZ"], J)
+    c = oracle.cols(P["X"], P["A"], P["a"], P["B"], P["dZ"], J, act)
     for k in ("H", "Y", "dH", "dA"):
         np.testing.assert_allclose(c[k], full[k][:, J], rtol=1e-14, atol=1e-15, err_msg=k)
     np.testing.assert_allclose(c["da"], full["da"][J], rtol=1e-14, atol=1e-15)
@@ -305,17 +329,18 @@ def test_rows_and_cols_match_full():
 
 # ------------------------------------------------ torch float64 cross-check
 
-def test_torch_float64_autograd():
-    """An independent implementation: torch CPU float64, exact GeLU, autograd."""
+@pytest.mark.parametrize("act", [0, 1])
+def test_torch_float64_autograd(act):
+    """An independent implementation: torch CPU float64, exact or tanh GeLU, autograd."""
     torch = pytest.importorskip("torch")
     rng = np.random.default_rng(7)
     T, h, F = 16, 8, 32
     P = _rand_problem(rng, T, h, F)
-    got = _all_outputs(oracle.default(), P)
+    got = _all_outputs(oracle.default(), P, act)
     t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=k != "dZ") for k, v in P.items()}
     Hh = t["X"] @ t["A"] + t["a"]
     Hh.retain_grad()
-    Yy = torch.nn.functional.gelu(Hh, approximate="none")
+    Yy = torch.nn.functional.gelu(Hh, approximate="tanh" if act else "none")
     Zz = Yy @ t["B"] + t["b"]
     (Zz * t["dZ"]).sum().backward()
     ref = dict(H=Hh, Y=Yy, Z=Zz, dH=Hh.grad, dX=t["X"].grad, dA=t["A"].grad, da=t["a"].grad,
@@ -338,6 +363,8 @@ MUTANTS = {
     "transposed_operand": ("mm_nt(T, h, F, dH, A, dX);", "mm_nn(T, h, F, dH, A, dX, 0);"),
     # bias a dropped from the pre-activation
     "dropped_bias": ("H[t * F + f] += a[f];", "H[t * F + f] += 0.0 * a[f];"),
+    # wrong cubic coefficient in the tanh form
+    "wrong_tanh_constant": ("#define TPO_GELU_TANH_C 0.044715", "#define TPO_GELU_TANH_C 0.04"),
     # db summing the wrong tensor's columns
     "wrong_index": ("tpo_colsum(T, h, dZ, db);\n    mm_tn(F, h, T, Y, dZ, dB);",
                     "tpo_colsum(T, h, dZ, db);\n    mm_tn(F, h, T, H, dZ, dB);"),
@@ -347,13 +374,16 @@ MUTANTS = {
 def _catches(orc):
     checks = [check_hand_example, check_bruteforce, check_finite_differences, check_normal_table]
     for chk in checks:
-        try:
-            if chk is check_bruteforce:
-                chk(orc, shapes=[(3, 2, 4), (5, 4, 12)])
-            else:
-                chk(orc)
-        except AssertionError:
-            return True
+        for act in (0, 1):
+            try:
+                if chk is check_bruteforce:
+                    chk(orc, shapes=[(3, 2, 4), (5, 4, 12)], act=act)
+                elif chk is check_finite_differences:
+                    chk(orc, act=act)
+                elif act == 0:
+                    chk(orc)
+            except AssertionError:
+                return True
     return False
 
 
