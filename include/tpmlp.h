@@ -51,6 +51,12 @@ typedef enum tpmlp_status {
  * FFMA throughout (no TF32). */
 typedef enum tpmlp_dtype { TPMLP_BF16 = 0, TPMLP_FP32 = 1 } tpmlp_dtype;
 
+/* Activation of the block. TPMLP_GELU_ERF is the exact GeLU x·Φ(x), the form
+ * tp_mlp_fwd and tp_mlp_bwd use (the pages name the activation only as
+ * "gelu"). TPMLP_GELU_TANH is the tanh approximation
+ * ½·x·(1 + tanh(√(2/π)·(x + 0.044715·x³))) (Hendrycks & Gimpel, 2016). */
+typedef enum tpmlp_activation { TPMLP_GELU_ERF = 0, TPMLP_GELU_TANH = 1 } tpmlp_activation;
+
 /* Bytes of device workspace that tp_mlp_fwd and tp_mlp_bwd need for these
  * sizes under the current split policy (the larger of the two calls' needs).
  * Returns 0 for invalid sizes. Holds the fp32 shard partials of the two
@@ -93,6 +99,20 @@ tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void
                         int p, tpmlp_dtype dt, void* workspace, size_t workspace_bytes,
                         void* stream);
 
+/* tp_mlp_fwd and tp_mlp_bwd with a selectable activation (GeLU in the
+ * forward, its derivative in the backward); same arguments, requirements
+ * and workspace, plus `act`. The backward must use the forward's `act`.
+ * Returns TPMLP_ERR_INVALID for an unknown `act`. */
+tpmlp_status tp_mlp_fwd_ex(const void* X, const void* A, const void* a, const void* B,
+                           const void* b, void* H, void* Y, void* Z, int64_t T, int64_t h,
+                           int64_t F, int p, tpmlp_dtype dt, tpmlp_activation act, void* workspace,
+                           size_t workspace_bytes, void* stream);
+tpmlp_status tp_mlp_bwd_ex(const void* dZ, const void* X, const void* A, const void* B,
+                           const void* H, const void* Y, void* dX, float* dA, float* da, float* dB,
+                           float* db, void* dH, int64_t T, int64_t h, int64_t F, int p,
+                           tpmlp_dtype dt, tpmlp_activation act, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* tpmlp_strerror(tpmlp_status s);
 
@@ -133,13 +153,16 @@ tpmlp_status tpmlp_wait_selftest(uint64_t limit_ns, void* stream);
 uint64_t tpmlp_launch_count(void);
 
 /* Evaluates GeLU(x[i]) into y[i] and GeLU′(x[i]) into dy[i] (fp32 device
- * arrays of n elements) with one of the two forms the kernels use, so the
- * approximation can be checked against CUDA's functions:
- *   form 0: the tensor-core epilogues' form, Φ(x) from the rational erf
- *           approximation of C. Hastings (Abramowitz & Stegun, Handbook of
- *           Mathematical Functions, eq. 7.1.26, |error| ≤ 1.5e−7) sharing
- *           exp(−x²/2) with φ(x);
- *   form 1: the plain path's form through CUDA's erff and expf.
+ * arrays of n elements) with one of the forms the kernels use, so the
+ * approximations can be checked against CUDA's functions:
+ *   form 0: exact GeLU as the tensor-core epilogues compute it, Φ(x) from
+ *           the rational erf approximation of C. Hastings (Abramowitz &
+ *           Stegun, Handbook of Mathematical Functions, eq. 7.1.26,
+ *           |error| ≤ 1.5e−7) sharing exp(−x²/2) with φ(x);
+ *   form 1: exact GeLU through CUDA's erff and expf (the plain path);
+ *   form 2: the tanh approximation as the tensor-core epilogues compute it,
+ *           tanh u = 1 − 2/(1 + exp(2u));
+ *   form 3: the tanh approximation through CUDA's tanhf (the plain path).
  * Returns TPMLP_ERR_INVALID for n < 0, null pointers or another form. */
 tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t n, int form,
                                    void* stream);

@@ -17,10 +17,12 @@ from .build import LIB as _LIB_PATH
 
 OK, ERR_INVALID, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(7)
 BF16, FP32 = 0, 1
+ACTIVATIONS = {"gelu": 0, "gelu_tanh": 1}
 
 # The entry points include/tpmlp.h declares, in declaration order.
 EXPORTS = (
-    "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tpmlp_strerror",
+    "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tp_mlp_fwd_ex", "tp_mlp_bwd_ex",
+    "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
@@ -55,6 +57,12 @@ def lib() -> ctypes.CDLL:
             L.tp_mlp_fwd.restype = ctypes.c_int
             L.tp_mlp_bwd.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
             L.tp_mlp_bwd.restype = ctypes.c_int
+            L.tp_mlp_fwd_ex.argtypes = [vp] * 8 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, vp, sz, vp]
+            L.tp_mlp_fwd_ex.restype = ctypes.c_int
+            L.tp_mlp_bwd_ex.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                    ctypes.c_int, vp, sz, vp]
+            L.tp_mlp_bwd_ex.restype = ctypes.c_int
             L.tpmlp_strerror.argtypes = [ctypes.c_int]
             L.tpmlp_strerror.restype = ctypes.c_char_p
             L.tpmlp_last_device_status.argtypes = [vp]
@@ -140,11 +148,20 @@ def _workspace(T, h, F, p, dtype, device, workspace):
     return workspace, workspace.numel() * workspace.element_size()
 
 
-def forward(X, A, a, B, b, p: int, *, out=None, workspace=None, stream=None):
+def _act_code(activation: str) -> int:
+    try:
+        return ACTIVATIONS[activation]
+    except KeyError:
+        raise ValueError(f"activation must be one of {sorted(ACTIVATIONS)}") from None
+
+
+def forward(X, A, a, B, b, p: int, *, out=None, workspace=None, stream=None,
+            activation: str = "gelu"):
     """H, Y, Z of Z = GeLU(X·A + a)·B + b with A, B split into p shards.
 
     X: T×h, A: h×F, a: F or None, B: F×h, b: h or None, all bf16 (or all
-    fp32) CUDA tensors. Returns (H, Y, Z); `out` may supply them."""
+    fp32) CUDA tensors. Returns (H, Y, Z); `out` may supply them.
+    activation: "gelu" (exact, x·Φ(x)) or "gelu_tanh" (tanh approximation)."""
     T, h = X.shape
     F = A.shape[1]
     dt, dev = X.dtype, X.device
@@ -165,15 +182,17 @@ def forward(X, A, a, B, b, p: int, *, out=None, workspace=None, stream=None):
         _need(Y, "Y", (T, F), dt, dev)
         _need(Z, "Z", (T, h), dt, dev)
     ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
-    st = lib().tp_mlp_fwd(_ptr(X), _ptr(A), _ptr(a), _ptr(B), _ptr(b), _ptr(H), _ptr(Y), _ptr(Z),
-                          T, h, F, int(p), _dtype_code(X), _ptr(ws), ws_bytes,
-                          _stream_ptr(dev, stream))
-    _check(st, "tp_mlp_fwd")
+    st = lib().tp_mlp_fwd_ex(_ptr(X), _ptr(A), _ptr(a), _ptr(B), _ptr(b), _ptr(H), _ptr(Y),
+                             _ptr(Z), T, h, F, int(p), _dtype_code(X), _act_code(activation),
+                             _ptr(ws), ws_bytes, _stream_ptr(dev, stream))
+    _check(st, "tp_mlp_fwd_ex")
     return H, Y, Z
 
 
-def backward(dZ, X, A, B, H, Y, p: int, *, out=None, workspace=None, stream=None):
-    """Gradients of the block for upstream gradient dZ (T×h).
+def backward(dZ, X, A, B, H, Y, p: int, *, out=None, workspace=None, stream=None,
+             activation: str = "gelu"):
+    """Gradients of the block for upstream gradient dZ (T×h); `activation`
+    must be the forward's.
 
     Returns a dict: dX (T×h, input dtype), dA (h×F, fp32), da (F, fp32),
     dB (F×h, fp32), db (h, fp32), dH (T×F, input dtype)."""
@@ -195,11 +214,11 @@ def backward(dZ, X, A, B, H, Y, p: int, *, out=None, workspace=None, stream=None
                          ("dB", (F, h), f32), ("db", (h,), f32), ("dH", (T, F), dt)):
         _need(out[name], name, shp, d, dev)
     ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
-    st = lib().tp_mlp_bwd(_ptr(dZ), _ptr(X), _ptr(A), _ptr(B), _ptr(H), _ptr(Y), _ptr(out["dX"]),
-                          _ptr(out["dA"]), _ptr(out["da"]), _ptr(out["dB"]), _ptr(out["db"]),
-                          _ptr(out["dH"]), T, h, F, int(p), _dtype_code(X), _ptr(ws), ws_bytes,
-                          _stream_ptr(dev, stream))
-    _check(st, "tp_mlp_bwd")
+    st = lib().tp_mlp_bwd_ex(_ptr(dZ), _ptr(X), _ptr(A), _ptr(B), _ptr(H), _ptr(Y),
+                             _ptr(out["dX"]), _ptr(out["dA"]), _ptr(out["da"]), _ptr(out["dB"]),
+                             _ptr(out["db"]), _ptr(out["dH"]), T, h, F, int(p), _dtype_code(X),
+                             _act_code(activation), _ptr(ws), ws_bytes, _stream_ptr(dev, stream))
+    _check(st, "tp_mlp_bwd_ex")
     return out
 
 
@@ -262,8 +281,10 @@ def profile_collect() -> dict:
 
 
 def eval_activation(x: torch.Tensor, form: int):
-    """(GeLU(x), GeLU′(x)) of a CUDA fp32 tensor with the kernels' form 0
-    (Hastings erf, tensor-core epilogues) or 1 (CUDA erff, plain path)."""
+    """(GeLU(x), GeLU′(x)) of a CUDA fp32 tensor with one of the kernels'
+    forms: 0 exact GeLU as the tensor-core epilogues compute it (Hastings
+    erf), 1 exact GeLU through CUDA's erff, 2 tanh form as the tensor-core
+    epilogues compute it, 3 tanh form through CUDA's tanhf."""
     if not x.is_cuda or x.dtype != torch.float32 or not x.is_contiguous():
         raise ValueError("x must be a contiguous CUDA float32 tensor")
     y = torch.empty_like(x)

@@ -174,15 +174,21 @@ __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restri
     }
 }
 
-// GeLU and GeLU′ of n values with either form the library uses:
-// form 0 = the tensor-core epilogues' (Hastings erf), 1 = CUDA's erff/expf.
+// GeLU and GeLU′ of n values with each form the library uses:
+// 0 = exact GeLU as in the tensor-core epilogues (Hastings erf), 1 = exact
+// GeLU through CUDA's erff/expf, 2 = tanh form as in the tensor-core
+// epilogues (exp-based tanh), 3 = tanh form through CUDA's tanhf.
 __global__ void eval_activation_kernel(const float* __restrict__ x, float* __restrict__ y,
                                        float* __restrict__ dy, int64_t n, int form) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float v = x[i];
-        y[i] = form == 0 ? gelu_fast(v) : gelu_f32(v);
-        dy[i] = form == 0 ? gelu_grad_fast(v) : gelu_grad_f32(v);
+        switch (form) {
+            case 0: y[i] = gelu_fast(v); dy[i] = gelu_grad_fast(v); break;
+            case 1: y[i] = gelu_f32(v); dy[i] = gelu_grad_f32(v); break;
+            case 2: y[i] = gelu_tanh_fast(v); dy[i] = gelu_tanh_grad_fast(v); break;
+            default: y[i] = gelu_tanh_f32(v); dy[i] = gelu_tanh_grad_f32(v); break;
+        }
     }
 }
 

@@ -29,10 +29,22 @@
 namespace tpmlp {
 
 enum EpiKind : int {
-    EPI_GELU = 0,       // out0 = H = acc + bias (bf16), out1 = Y = GeLU(H) (bf16)
-    EPI_BIAS = 1,       // out0 = acc + bias (element type); bias may be null
-    EPI_DGELU = 2,      // out0 = dH = acc · GeLU′(aux) (bf16), aux = saved H (bf16)
-    EPI_F32 = 3,        // out0 (fp32) + split · split_stride = acc
+    EPI_GELU = 0,        // out0 = H = acc + bias (bf16), out1 = Y = GeLU(H) (bf16)
+    EPI_BIAS = 1,        // out0 = acc + bias (element type); bias may be null
+    EPI_DGELU = 2,       // out0 = dH = acc · GeLU′(aux) (bf16), aux = saved H (bf16)
+    EPI_F32 = 3,         // out0 (fp32) + split · split_stride = acc
+    EPI_GELU_TANH = 4,   // as EPI_GELU with the tanh approximation of GeLU
+    EPI_DGELU_TANH = 5,  // as EPI_DGELU with the tanh approximation's derivative
+};
+
+// Epilogue classes: activation forward (two outputs), activation backward
+// (reads the saved pre-activation), and the tanh forms of both.
+template <int EPI>
+struct EpiTraits {
+    static constexpr bool kAct = (EPI == EPI_GELU || EPI == EPI_GELU_TANH);
+    static constexpr bool kDAct = (EPI == EPI_DGELU || EPI == EPI_DGELU_TANH);
+    static constexpr bool kTanh = (EPI == EPI_GELU_TANH || EPI == EPI_DGELU_TANH);
+    static constexpr bool kBias = (EPI == EPI_BIAS) || kAct;
 };
 
 struct GemmArgs {
@@ -132,6 +144,52 @@ __device__ __forceinline__ float gelu_grad_fast(float x) {
     return fmaf(x * 0.39894228040143268f, g, cdf);
 }
 
+// The tanh approximation of GeLU, ½·x·(1 + tanh u), u = √(2/π)·(x + 0.044715·x³),
+// with tanh u = 1 − 2 / (1 + exp(2u)) (one exponential and one reciprocal;
+// exp(2u) = ∞ gives tanh u = 1 and exp(2u) = 0 gives −1, as they should).
+__device__ __forceinline__ float tanh_via_exp(float u) {
+    return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * u));
+}
+
+__device__ __forceinline__ float gelu_tanh_fast(float x) {
+    const float u = 0.79788456080286536f * x * fmaf(0.044715f * x, x, 1.0f);
+    return 0.5f * x * (1.0f + tanh_via_exp(u));
+}
+
+// ½(1 + tanh u) + ½·x·(1 − tanh² u)·√(2/π)·(1 + 3·0.044715·x²)
+__device__ __forceinline__ float gelu_tanh_grad_fast(float x) {
+    const float u = 0.79788456080286536f * x * fmaf(0.044715f * x, x, 1.0f);
+    const float th = tanh_via_exp(u);
+    const float du = 0.79788456080286536f * fmaf(0.134145f * x, x, 1.0f);
+    return fmaf(0.5f * x * du, fmaf(-th, th, 1.0f), 0.5f * (1.0f + th));
+}
+
+// The same two functions through CUDA's tanhf (the plain path).
+__device__ __forceinline__ float gelu_tanh_f32(float x) {
+    const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
+    return 0.5f * x * (1.0f + tanhf(u));
+}
+
+__device__ __forceinline__ float gelu_tanh_grad_f32(float x) {
+    const float u = 0.79788456080286536f * (x + 0.044715f * x * x * x);
+    const float th = tanhf(u);
+    const float du = 0.79788456080286536f * (1.0f + 0.134145f * x * x);
+    return 0.5f * (1.0f + th) + 0.5f * x * (1.0f - th * th) * du;
+}
+
+// Activation of the tensor-core epilogues for epilogue kind EPI.
+template <int EPI>
+__device__ __forceinline__ float act_fast(float x) {
+    if constexpr (EpiTraits<EPI>::kTanh) return gelu_tanh_fast(x);
+    else return gelu_fast(x);
+}
+
+template <int EPI>
+__device__ __forceinline__ float act_grad_fast(float x) {
+    if constexpr (EpiTraits<EPI>::kTanh) return gelu_tanh_grad_fast(x);
+    else return gelu_grad_fast(x);
+}
+
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
@@ -186,7 +244,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             float v[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[8 * q + i]);
-            if constexpr (EPI == EPI_GELU || EPI == EPI_BIAS) {
+            if constexpr (EpiTraits<EPI>::kBias) {
                 if (g.bias != nullptr && c < g.N) {
                     float bb[8];
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.bias + c)), bb);
@@ -194,22 +252,22 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
                     for (int i = 0; i < 8; ++i) v[i] += bb[i];
                 }
             }
-            if constexpr (EPI == EPI_DGELU) {
+            if constexpr (EpiTraits<EPI>::kDAct) {
                 float hh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
                 if (row < g.M && c < g.N)
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= gelu_grad_fast(hh[i]);
+                for (int i = 0; i < 8; ++i) v[i] *= act_grad_fast<EPI>(hh[i]);
             }
             o0[q].x = pack_bf16x2(v[0], v[1]);
             o0[q].y = pack_bf16x2(v[2], v[3]);
             o0[q].z = pack_bf16x2(v[4], v[5]);
             o0[q].w = pack_bf16x2(v[6], v[7]);
-            if constexpr (EPI == EPI_GELU) {
-                o1[q].x = pack_bf16x2(gelu_fast(v[0]), gelu_fast(v[1]));
-                o1[q].y = pack_bf16x2(gelu_fast(v[2]), gelu_fast(v[3]));
-                o1[q].z = pack_bf16x2(gelu_fast(v[4]), gelu_fast(v[5]));
-                o1[q].w = pack_bf16x2(gelu_fast(v[6]), gelu_fast(v[7]));
+            if constexpr (EpiTraits<EPI>::kAct) {
+                o1[q].x = pack_bf16x2(act_fast<EPI>(v[0]), act_fast<EPI>(v[1]));
+                o1[q].y = pack_bf16x2(act_fast<EPI>(v[2]), act_fast<EPI>(v[3]));
+                o1[q].z = pack_bf16x2(act_fast<EPI>(v[4]), act_fast<EPI>(v[5]));
+                o1[q].w = pack_bf16x2(act_fast<EPI>(v[6]), act_fast<EPI>(v[7]));
             }
         }
         if (lane == 0) bulk_wait_read0();
@@ -218,13 +276,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
         for (int q = 0; q < 4; ++q) {
             const uint32_t a = lane * 64 + ((q ^ ((lane >> 1) & 3)) << 4);
             st_shared_v4(slot + a, o0[q]);
-            if constexpr (EPI == EPI_GELU) st_shared_v4(slot + 2048 + a, o1[q]);
+            if constexpr (EpiTraits<EPI>::kAct) st_shared_v4(slot + 2048 + a, o1[q]);
         }
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && any) {
             tma_store_3d(tmO0, slot, col0, row0, 0);
-            if constexpr (EPI == EPI_GELU) tma_store_3d(tmO1, slot + 2048, col0, row0, 0);
+            if constexpr (EpiTraits<EPI>::kAct) tma_store_3d(tmO1, slot + 2048, col0, row0, 0);
             bulk_commit();
         }
     }
@@ -265,7 +323,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     const uint32_t partner_slot = smem_u32(sEpi + (4 * half + quad) * kEpiSlotBytes);
     if (lane == 0 && !relay) {
         tma_prefetch_desc(tmO0);
-        if (EPI == EPI_GELU) tma_prefetch_desc(tmO1);
+        if (EpiTraits<EPI>::kAct) tma_prefetch_desc(tmO1);
     }
     uint32_t xcount = 0;
     int local = 0;

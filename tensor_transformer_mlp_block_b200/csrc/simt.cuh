@@ -68,12 +68,16 @@ __global__ void __launch_bounds__(256) simt_gemm_kernel(const SimtArgs g) {
         static_cast<float*>(g.out0)[off] = acc;
     } else {
         float v = acc;
-        if constexpr (EPI == EPI_GELU || EPI == EPI_BIAS) {
+        if constexpr (EpiTraits<EPI>::kBias) {
             if (g.bias != nullptr) v += ld_f32<T>(static_cast<const T*>(g.bias) + n);
         }
-        if constexpr (EPI == EPI_DGELU) v *= gelu_grad_f32(ld_f32<T>(static_cast<const T*>(g.aux) + off));
+        if constexpr (EpiTraits<EPI>::kDAct) {
+            const float hv = ld_f32<T>(static_cast<const T*>(g.aux) + off);
+            v *= EpiTraits<EPI>::kTanh ? gelu_tanh_grad_f32(hv) : gelu_grad_f32(hv);
+        }
         static_cast<T*>(g.out0)[off] = from_f32<T>(v);
-        if constexpr (EPI == EPI_GELU) static_cast<T*>(g.out1)[off] = from_f32<T>(gelu_f32(v));
+        if constexpr (EpiTraits<EPI>::kAct)
+            static_cast<T*>(g.out1)[off] = from_f32<T>(EpiTraits<EPI>::kTanh ? gelu_tanh_f32(v) : gelu_f32(v));
     }
 }
 

@@ -126,7 +126,7 @@ template <int EPI>
 bool make_out_maps(CUtensorMap* o0, CUtensorMap* o1, const GemmArgs& g, int M, int N, int splits) {
     const bool f32 = (EPI == EPI_F32);
     if (!make_out_map(o0, g.out0, f32 ? splits : 1, M, N, f32)) return false;
-    if (EPI == EPI_GELU) return make_out_map(o1, g.out1, 1, M, N, false);
+    if (EpiTraits<EPI>::kAct) return make_out_map(o1, g.out1, 1, M, N, false);
     *o1 = *o0;
     return true;
 }
@@ -188,9 +188,11 @@ tpmlp_status timed(int kind, double flops, double bytes, cudaStream_t st, Fn&& f
 
 // ------------------------------------------------------ tensor-core launches
 
+// Index of a tensor-core kernel instantiation (0..47) for per-device caches.
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 constexpr int kernel_id() {
-    return (EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) + (BN == 128 ? 16 : 0) + (RELAY ? 32 : 0);
+    static_assert(BN == 256, "the launchers use 256-column tiles");
+    return (EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2 + (RELAY ? 1 : 0);
 }
 
 // D[M, N] = Aop·Bop with Aop stored [M][K] (A_MN = false) or [K][M], Bop
@@ -298,9 +300,9 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
 template <int EPI>
 double gemm_bytes(double M, double N, double K, int splits) {
     double b = 2.0 * (M * K + K * N);
-    if (EPI == EPI_GELU) b += 2.0 * 2.0 * M * N;
+    if (EpiTraits<EPI>::kAct) b += 2.0 * 2.0 * M * N;
     if (EPI == EPI_BIAS) b += 2.0 * M * N;
-    if (EPI == EPI_DGELU) b += 2.0 * 2.0 * M * N;
+    if (EpiTraits<EPI>::kDAct) b += 2.0 * 2.0 * M * N;
     if (EPI == EPI_F32) b += 4.0 * M * N * splits;
     return b;
 }
@@ -324,7 +326,7 @@ tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, i
                      GemmArgs g, cudaStream_t st) {
     return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K, splits), st, [&] {
         const int k_per_unit = splits > 1 ? K / splits : K;
-        const int threshold = (EPI == EPI_GELU || EPI == EPI_DGELU) ? 3072 : 2048;
+        const int threshold = (EpiTraits<EPI>::kAct || EpiTraits<EPI>::kDAct) ? 3072 : 2048;
         if (k_per_unit < threshold)
             return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, splits, g, st);
         return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, splits, g, st);
@@ -487,22 +489,11 @@ tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype d
     return TPMLP_OK;
 }
 
-}  // namespace
-}  // namespace tpmlp
-
-using namespace tpmlp;
-
-extern "C" {
-
-size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt) {
-    Plan pl;
-    if (!make_plan(T, h, F, p, dt, &pl)) return 0;
-    return pl.total;
-}
-
-tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void* B, const void* b,
-                        void* H, void* Y, void* Z, int64_t T, int64_t h, int64_t F, int p,
-                        tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+// Forward with activation epilogue EPI_ACT (EPI_GELU or EPI_GELU_TANH).
+template <int EPI_ACT>
+tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B, const void* b,
+                      void* H, void* Y, void* Z, int64_t T, int64_t h, int64_t F, int p,
+                      tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
     cudaGetLastError();  // start from a clean (non-sticky) error state
     Plan pl;
     TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes));
@@ -520,7 +511,7 @@ tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void*
         g1.out1 = Y;
         g1.ld_out = F;
         g1.bias = static_cast<const __nv_bfloat16*>(a);
-        TPMLP_TRY((gemm_tc<256, false, true, EPI_GELU>(K_F1, X, A, iT, iF, ih, 1, g1, st)));
+        TPMLP_TRY((gemm_tc<256, false, true, EPI_ACT>(K_F1, X, A, iT, iF, ih, 1, g1, st)));
         // F2: Z = Σ_i Y_i·B_i + b. Aop = Y [T][F] (K-major), Bop = B [F][h] (MN-major).
         GemmArgs g2{};
         if (pl.splits == 1) {
@@ -550,19 +541,21 @@ tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void*
     s2.B = B; s2.sbk = h; s2.sbn = 1;
     s2.out0 = Z; s2.ld_out = h; s2.bias = b;
     if (dt == TPMLP_FP32) {
-        TPMLP_TRY((gemm_simt<float, EPI_GELU>(K_F1, s1, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_ACT>(K_F1, s1, st)));
         TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_F2, s2, st)));
     } else {
-        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_GELU>(K_F1, s1, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_ACT>(K_F1, s1, st)));
         TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_F2, s2, st)));
     }
     return TPMLP_OK;
 }
 
-tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void* B, const void* H,
-                        const void* Y, void* dX, float* dA, float* da, float* dB, float* db,
-                        void* dH, int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
-                        void* workspace, size_t workspace_bytes, void* stream) {
+// Backward with activation-derivative epilogue EPI_DACT (EPI_DGELU or EPI_DGELU_TANH).
+template <int EPI_DACT>
+tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* B, const void* H,
+                      const void* Y, void* dX, float* dA, float* da, float* dB, float* db,
+                      void* dH, int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
+                      void* workspace, size_t workspace_bytes, void* stream) {
     cudaGetLastError();
     Plan pl;
     TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes));
@@ -593,7 +586,7 @@ tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
-        TPMLP_TRY((gemm_tc<256, false, false, EPI_DGELU>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
         // da = 1ᵀ·dH
         TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
@@ -649,20 +642,79 @@ tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void
     s5.out0 = dX; s5.ld_out = h;
     if (dt == TPMLP_FP32) {
         TPMLP_TRY(colsum(K_B1_DB, static_cast<const float*>(dZ), T, h, pl.chunks, cs_h, db, st));
-        TPMLP_TRY((gemm_simt<float, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY((gemm_simt<float, EPI_DACT>(K_B2, s2, st)));
         TPMLP_TRY(colsum(K_B2_DA, static_cast<const float*>(dH), T, F, pl.chunks, cs_f, da, st));
         TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B3, s3, st)));
         TPMLP_TRY((gemm_simt<float, EPI_F32>(K_B4, s4, st)));
         TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_B5, s5, st)));
     } else {
         TPMLP_TRY(colsum(K_B1_DB, static_cast<const __nv_bfloat16*>(dZ), T, h, pl.chunks, cs_h, db, st));
-        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_DGELU>(K_B2, s2, st)));
+        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_DACT>(K_B2, s2, st)));
         TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
         TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B3, s3, st)));
         TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_B4, s4, st)));
         TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_B5, s5, st)));
     }
     return TPMLP_OK;
+}
+
+}  // namespace
+}  // namespace tpmlp
+
+using namespace tpmlp;
+
+extern "C" {
+
+size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt) {
+    Plan pl;
+    if (!make_plan(T, h, F, p, dt, &pl)) return 0;
+    return pl.total;
+}
+
+tpmlp_status tp_mlp_fwd(const void* X, const void* A, const void* a, const void* B, const void* b,
+                        void* H, void* Y, void* Z, int64_t T, int64_t h, int64_t F, int p,
+                        tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+    return fwd_impl<EPI_GELU>(X, A, a, B, b, H, Y, Z, T, h, F, p, dt, workspace, workspace_bytes,
+                              stream);
+}
+
+tpmlp_status tp_mlp_fwd_ex(const void* X, const void* A, const void* a, const void* B,
+                           const void* b, void* H, void* Y, void* Z, int64_t T, int64_t h,
+                           int64_t F, int p, tpmlp_dtype dt, tpmlp_activation act, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    switch (act) {
+        case TPMLP_GELU_ERF:
+            return fwd_impl<EPI_GELU>(X, A, a, B, b, H, Y, Z, T, h, F, p, dt, workspace,
+                                      workspace_bytes, stream);
+        case TPMLP_GELU_TANH:
+            return fwd_impl<EPI_GELU_TANH>(X, A, a, B, b, H, Y, Z, T, h, F, p, dt, workspace,
+                                           workspace_bytes, stream);
+    }
+    return TPMLP_ERR_INVALID;
+}
+
+tpmlp_status tp_mlp_bwd(const void* dZ, const void* X, const void* A, const void* B, const void* H,
+                        const void* Y, void* dX, float* dA, float* da, float* dB, float* db,
+                        void* dH, int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    return bwd_impl<EPI_DGELU>(dZ, X, A, B, H, Y, dX, dA, da, dB, db, dH, T, h, F, p, dt, workspace,
+                               workspace_bytes, stream);
+}
+
+tpmlp_status tp_mlp_bwd_ex(const void* dZ, const void* X, const void* A, const void* B,
+                           const void* H, const void* Y, void* dX, float* dA, float* da, float* dB,
+                           float* db, void* dH, int64_t T, int64_t h, int64_t F, int p,
+                           tpmlp_dtype dt, tpmlp_activation act, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+    switch (act) {
+        case TPMLP_GELU_ERF:
+            return bwd_impl<EPI_DGELU>(dZ, X, A, B, H, Y, dX, dA, da, dB, db, dH, T, h, F, p, dt,
+                                       workspace, workspace_bytes, stream);
+        case TPMLP_GELU_TANH:
+            return bwd_impl<EPI_DGELU_TANH>(dZ, X, A, B, H, Y, dX, dA, da, dB, db, dH, T, h, F, p,
+                                            dt, workspace, workspace_bytes, stream);
+    }
+    return TPMLP_ERR_INVALID;
 }
 
 const char* tpmlp_strerror(tpmlp_status s) {
@@ -708,7 +760,7 @@ uint64_t tpmlp_launch_count(void) { return g_launches.load(); }
 tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t n, int form,
                                    void* stream) {
     cudaGetLastError();
-    if (n < 0 || (form != 0 && form != 1)) return TPMLP_ERR_INVALID;
+    if (n < 0 || form < 0 || form > 3) return TPMLP_ERR_INVALID;
     if (n == 0) return TPMLP_OK;
     if (!x || !y || !dy) return TPMLP_ERR_INVALID;
     int64_t blocks = (n + 255) / 256;

@@ -43,12 +43,12 @@ def _u(key: str, dtype: str) -> float:
     return UNIT_ROUNDOFF[dtype] if key.split("[")[0] in STORED else 0.0
 
 
-def run_gpu(inp: dict, p: int, device="cuda:0"):
+def run_gpu(inp: dict, p: int, device="cuda:0", activation: str = "gelu"):
     """Forward + backward on the GPU through the binding. Returns CPU tensors."""
     from tensor_transformer_mlp_block_b200 import binding
     d = {k: v.to(device) for k, v in inp.items()}
-    H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p)
-    g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, p)
+    H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p, activation=activation)
+    g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, p, activation=activation)
     torch.cuda.synchronize()
     st = binding.last_device_status()
     assert st == 0, f"device status {st}"
@@ -56,11 +56,11 @@ def run_gpu(inp: dict, p: int, device="cuda:0"):
     return {k: v.cpu() for k, v in out.items()}
 
 
-def oracle_full(inp: dict):
-    """Full fp64 oracle on the rounded inputs."""
+def oracle_full(inp: dict, act: int = 0):
+    """Full fp64 oracle on the rounded inputs (act: 0 exact GeLU, 1 tanh form)."""
     n = {k: to_np(v) for k, v in inp.items()}
-    H, Y, Z = oracle.forward(n["X"], n["A"], n["a"], n["B"], n["b"])
-    g = oracle.backward(n["X"], n["A"], n["B"], H, Y, n["dZ"])
+    H, Y, Z = oracle.forward(n["X"], n["A"], n["a"], n["B"], n["b"], act)
+    g = oracle.backward(n["X"], n["A"], n["B"], H, Y, n["dZ"], act)
     return dict(H=H, Y=Y, Z=Z, **g)
 
 
@@ -75,16 +75,16 @@ def compare_full(gpu: dict, ref: dict, dtype: str, keys=None) -> dict:
     return errs
 
 
-def compare_sampled(gpu: dict, inp: dict, R, J, dtype: str) -> dict:
+def compare_sampled(gpu: dict, inp: dict, R, J, dtype: str, act: int = 0) -> dict:
     """Compare on token rows R and hidden columns J, each computed exactly by
     the oracle (rows: H, Y, Z, dH, dX; columns: H, Y, dH, dA, da, dB), plus
     db in full."""
     n = {k: to_np(v) for k, v in inp.items()}
     R = np.asarray(R)
     J = np.asarray(J)
-    r = oracle.rows(n["X"], n["A"], n["a"], n["B"], n["b"], n["dZ"], R)
+    r = oracle.rows(n["X"], n["A"], n["a"], n["B"], n["b"], n["dZ"], R, act)
     # the column subset needs only A[:, J], a[J], B[J, :]
-    c = oracle.cols(n["X"], n["A"][:, J], n["a"][J], n["B"][J, :], n["dZ"], np.arange(len(J)))
+    c = oracle.cols(n["X"], n["A"][:, J], n["a"][J], n["B"][J, :], n["dZ"], np.arange(len(J)), act)
     db = oracle.colsum(n["dZ"])
     tol = TOL[dtype]
     errs = {}

@@ -40,3 +40,20 @@ def test_fast_form_against_fp64_oracle():
     # exact special values of the form
     assert y0[np.where(xs == 0.0)[0][0]] == 0.0
     assert abs(d0[np.where(xs == 0.0)[0][0]] - 0.5) < 1e-7
+
+
+def test_tanh_forms_match_each_other_and_the_oracle():
+    """The tanh approximation as the tensor-core epilogues compute it (tanh
+    from one exponential) against CUDA's tanhf form and the fp64 oracle."""
+    x = _grid()
+    y2, d2 = binding.eval_activation(x.cuda(), 2)
+    y3, d3 = binding.eval_activation(x.cuda(), 3)
+    xa = x.abs().double().cuda()
+    assert torch.all((y2.double() - y3.double()).abs() <= 1e-6 * xa + 1e-30)
+    assert torch.all((d2.double() - d3.double()).abs() <= 2e-6 * (1 + xa))
+    y2, d2 = y2.cpu().double().numpy(), d2.cpu().double().numpy()
+    xs = x.double().numpy()
+    for i in np.linspace(0, len(xs) - 1, 4001).astype(int):
+        g, dg = oracle.gelu_tanh(xs[i]), oracle.gelu_tanh_grad(xs[i])
+        assert abs(y2[i] - g) <= 1e-6 * abs(xs[i]) + 1e-7 * abs(g) + 1e-37, (xs[i], y2[i], g)
+        assert abs(d2[i] - dg) <= 2e-6 * (1 + abs(xs[i])), (xs[i], d2[i], dg)

@@ -134,3 +134,44 @@ def test_named_config_gpt2_full():
     inp = make_inputs(cfg)
     gpu = run_gpu(inp, cfg.p)
     compare_full(gpu, oracle_full(inp), "bf16")
+
+
+@pytest.mark.parametrize("T,h,F,p", [(300, 200, 520, 2), (256, 128, 512, 4), (37, 12, 44, 2)])
+def test_gelu_tanh_variant(T, h, F, p):
+    """The tanh approximation (activation="gelu_tanh") against the oracle's
+    tanh form, on the tensor-core and the plain paths."""
+    inp = make_shape(T, h, F, "bf16", seed_offset=T + 7)
+    gpu = run_gpu(inp, p, activation="gelu_tanh")
+    compare_full(gpu, oracle_full(inp, act=1), "bf16")
+
+
+def test_gelu_tanh_variant_fp32():
+    cfg = configs.get("tiny")
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p, activation="gelu_tanh")
+    compare_full(gpu, oracle_full(inp, act=1), "fp32")
+
+
+def test_gelu_tanh_variant_7b_sampled():
+    """The tanh variant on the 7B-class workload, where the GeLU epilogues use
+    the relaying warps (K = 4096)."""
+    cfg = configs.get("7b")
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p, activation="gelu_tanh")
+    R = sample_indices(cfg.T, 32, seed=1234).numpy()
+    J = sample_indices(cfg.F, 48, seed=1235).numpy()
+    compare_sampled(gpu, inp, R, J, cfg.dtype, act=1)
+
+
+def test_activation_forms_differ_where_they_should():
+    """Exact and tanh forms give different Y (by up to ~5e-4·|x| scale), the
+    same shapes, and the backward refuses an unknown activation name."""
+    from tensor_transformer_mlp_block_b200 import binding
+    inp = make_shape(256, 128, 512, "bf16", seed_offset=3)
+    a = run_gpu(inp, 2)
+    b = run_gpu(inp, 2, activation="gelu_tanh")
+    assert torch.equal(a["H"], b["H"])
+    assert not torch.equal(a["Y"], b["Y"])
+    d = {k: v.cuda() for k, v in inp.items()}
+    with pytest.raises(ValueError):
+        binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], 2, activation="relu")
