@@ -33,6 +33,10 @@ from .oracle import (  # noqa: F401
     gelu_tanh,
     gelu_tanh_grad,
     get_threads,
+    linear_backward,
+    linear_backward_sharded,
+    linear_forward,
+    linear_forward_sharded,
     normal_cdf,
     normal_pdf,
     rows,

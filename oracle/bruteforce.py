@@ -57,3 +57,15 @@ def mlp(X, A, a, B, b, dZ, act: int = 0):
     dA = [[math.fsum(X[t][k] * dH[t][f] for t in range(T)) for f in range(F)] for k in range(h)]
     dX = [[math.fsum(dH[t][f] * A[k][f] for f in range(F)) for k in range(h)] for t in range(T)]
     return dict(H=H, Y=Y, Z=Z, dH=dH, dX=dX, dA=dA, da=da, dB=dB, db=db)
+
+
+def linear(X, W, bias, dY):
+    """Y = X·W + bias and its gradients (dX, dW, dbias) for upstream dY,
+    as nested lists; X: T×K, W: K×N, bias: N, dY: T×N."""
+    T, K, N = len(X), len(X[0]), len(W[0])
+    Y = [[math.fsum([X[t][k] * W[k][n] for k in range(K)] + [bias[n]]) for n in range(N)]
+         for t in range(T)]
+    db = [math.fsum(dY[t][n] for t in range(T)) for n in range(N)]
+    dW = [[math.fsum(X[t][k] * dY[t][n] for t in range(T)) for n in range(N)] for k in range(K)]
+    dX = [[math.fsum(dY[t][n] * W[k][n] for n in range(N)) for k in range(K)] for t in range(T)]
+    return dict(Y=Y, dX=dX, dW=dW, db=db)

@@ -62,6 +62,12 @@ def _bind(path: str):
     lib.tpo_backward_sharded_act.restype = _c
     lib.tpo_rows_act.argtypes = [_I64, _I64, _I64] + [_D] * 6 + [_I64, _P64] + [_D] * 5 + [_c]
     lib.tpo_cols_act.argtypes = [_I64, _I64, _I64] + [_D] * 5 + [_I64, _P64] + [_D] * 6 + [_c]
+    lib.tpo_linear_forward.argtypes = [_I64, _I64, _I64] + [_D] * 4
+    lib.tpo_linear_backward.argtypes = [_I64, _I64, _I64] + [_D] * 6
+    lib.tpo_linear_forward_sharded.argtypes = [_I64, _I64, _I64, _c, _c] + [_D] * 4
+    lib.tpo_linear_forward_sharded.restype = _c
+    lib.tpo_linear_backward_sharded.argtypes = [_I64, _I64, _I64, _c, _c] + [_D] * 6
+    lib.tpo_linear_backward_sharded.restype = _c
     return lib
 
 
@@ -194,6 +200,51 @@ class Oracle:
         return out
 
 
+    # ------------------------------------------------ tensor-parallel linear
+    def linear_forward(self, X, W, bias):
+        """Y = X·W + bias (unsplit). X: T×K, W: K×N, bias: N."""
+        X, W, bias = map(_in, (X, W, bias))
+        T, K = X.shape
+        N = W.shape[1]
+        assert W.shape == (K, N) and bias.shape == (N,)
+        Y = np.empty((T, N))
+        self._lib.tpo_linear_forward(T, K, N, *map(_ptr, (X, W, bias, Y)))
+        return Y
+
+    def linear_backward(self, X, W, dY):
+        """(dX, dW, dbias) of Y = X·W + bias (unsplit)."""
+        X, W, dY = map(_in, (X, W, dY))
+        T, K = X.shape
+        N = W.shape[1]
+        dX, dW, db = np.empty((T, K)), np.empty((K, N)), np.empty(N)
+        self._lib.tpo_linear_backward(T, K, N, *map(_ptr, (X, W, dY, dX, dW, db)))
+        return dX, dW, db
+
+    def linear_forward_sharded(self, X, W, bias, p: int, split: str):
+        """Y through the p-way partition; split = "columns" or "rows"."""
+        X, W, bias = map(_in, (X, W, bias))
+        T, K = X.shape
+        N = W.shape[1]
+        Y = np.empty((T, N))
+        rc = self._lib.tpo_linear_forward_sharded(T, K, N, int(p), {"columns": 0, "rows": 1}[split],
+                                                  *map(_ptr, (X, W, bias, Y)))
+        if rc != 0:
+            raise ValueError(f"p={p} does not divide the {split} dimension")
+        return Y
+
+    def linear_backward_sharded(self, X, W, dY, p: int, split: str):
+        X, W, dY = map(_in, (X, W, dY))
+        T, K = X.shape
+        N = W.shape[1]
+        dX, dW, db = np.empty((T, K)), np.empty((K, N)), np.empty(N)
+        rc = self._lib.tpo_linear_backward_sharded(T, K, N, int(p),
+                                                   {"columns": 0, "rows": 1}[split],
+                                                   *map(_ptr, (X, W, dY, dX, dW, db)))
+        if rc != 0:
+            raise ValueError(f"p={p} does not divide the {split} dimension")
+        return dX, dW, db
+
+
 def compile_variant(source_text: str, out_path: str) -> Oracle:
     """Compile a (possibly edited) copy of the oracle source and bind it.
     Used by the tests to plant mistakes in a throw-away build and check that
@@ -276,3 +327,19 @@ def rows(X, A, a, B, b, dZ, R, act=0):
 
 def cols(X, A, a, B, dZ, J, act=0):
     return default().cols(X, A, a, B, dZ, J, act)
+
+
+def linear_forward(X, W, bias):
+    return default().linear_forward(X, W, bias)
+
+
+def linear_backward(X, W, dY):
+    return default().linear_backward(X, W, dY)
+
+
+def linear_forward_sharded(X, W, bias, p, split):
+    return default().linear_forward_sharded(X, W, bias, p, split)
+
+
+def linear_backward_sharded(X, W, dY, p, split):
+    return default().linear_backward_sharded(X, W, dY, p, split)

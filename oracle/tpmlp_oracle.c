@@ -383,3 +383,113 @@ void tpo_cols(int64_t T, int64_t h, int64_t F, const double* X, const double* A,
               double* da_J, double* dB_J) {
     tpo_cols_act(T, h, F, X, A, a, B, dZ, nJ, J, H_J, Y_J, dH_J, dA_J, da_J, dB_J, 0);
 }
+
+/* ---------------------------------------------------------------------------
+ * Tensor-parallel linear layers (page "Megatron", section "张量并行 / 数学原理"
+ * for the two splits, section "Transformer层的张量并行实现" for their use in the
+ * attention layer: the QKV projection is split by columns, the output
+ * projection by rows). Unsplit, both compute
+ *
+ *   Y = X·W + 1·biasᵀ      X: T × K, W: K × N, Y: T × N
+ *   dbias = 1ᵀ·dY,  dW = Xᵀ·dY,  dX = dY·Wᵀ
+ *
+ * The _sharded forms follow the partition literally. Column split: shard i
+ * holds W_i = W[:, i·N/p : (i+1)·N/p] and bias_i; Y_i = X·W_i + bias_i side
+ * by side (no exchange); backward dW_i = Xᵀ·dY_i, dbias_i = 1ᵀ·dY_i and, X
+ * being replicated, dX = Σ_i dY_i·W_iᵀ over i = 1..p in order. Row split:
+ * shard i holds W_i = W[i·K/p : (i+1)·K/p, :] and the matching columns X_i
+ * of X; Y = Σ_i X_i·W_i (in order) + bias; backward dX_i = dY·W_iᵀ (no
+ * exchange), dW_i = X_iᵀ·dY, dbias = 1ᵀ·dY.
+ * ------------------------------------------------------------------------- */
+
+void tpo_linear_forward(int64_t T, int64_t K, int64_t N, const double* X, const double* W,
+                        const double* bias, double* Y) {
+    mm_nn(T, N, K, X, W, Y, 0);
+#pragma omp parallel for schedule(static)
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) Y[t * N + n] += bias[n];
+}
+
+void tpo_linear_backward(int64_t T, int64_t K, int64_t N, const double* X, const double* W,
+                         const double* dY, double* dX, double* dW, double* dbias) {
+    tpo_colsum(T, N, dY, dbias);
+    mm_tn(K, N, T, X, dY, dW);
+    mm_nt(T, K, N, dY, W, dX);
+}
+
+/* split: 0 = columns, 1 = rows. Returns -1 if p does not divide the split
+ * dimension (N for columns, K for rows). */
+int tpo_linear_forward_sharded(int64_t T, int64_t K, int64_t N, int p, int split, const double* X,
+                               const double* W, const double* bias, double* Y) {
+    if (p < 1) return -1;
+    if (split == 0) {
+        if (N % p != 0) return -1;
+        const int64_t Np = N / p;
+        double* Yi = (double*)malloc((size_t)(T * Np) * sizeof(double));
+        for (int i = 0; i < p; ++i) {
+            double* Wi = col_block(K, N, W, i * Np, Np);
+            mm_nn(T, Np, K, X, Wi, Yi, 0);
+            for (int64_t t = 0; t < T; ++t)
+                for (int64_t n = 0; n < Np; ++n) Y[t * N + i * Np + n] = Yi[t * Np + n] + bias[i * Np + n];
+            free(Wi);
+        }
+        free(Yi);
+        return 0;
+    }
+    if (K % p != 0) return -1;
+    const int64_t Kp = K / p;
+    double* Pi = (double*)malloc((size_t)(T * N) * sizeof(double));
+    memset(Y, 0, (size_t)(T * N) * sizeof(double));
+    for (int i = 0; i < p; ++i) {
+        double* Xi = col_block(T, K, X, i * Kp, Kp);
+        mm_nn(T, N, Kp, Xi, W + (int64_t)i * Kp * N, Pi, 0);
+        for (int64_t e = 0; e < T * N; ++e) Y[e] += Pi[e];
+        free(Xi);
+    }
+    for (int64_t t = 0; t < T; ++t)
+        for (int64_t n = 0; n < N; ++n) Y[t * N + n] += bias[n];
+    free(Pi);
+    return 0;
+}
+
+int tpo_linear_backward_sharded(int64_t T, int64_t K, int64_t N, int p, int split, const double* X,
+                                const double* W, const double* dY, double* dX, double* dW,
+                                double* dbias) {
+    if (p < 1) return -1;
+    tpo_colsum(T, N, dY, dbias);
+    if (split == 0) {
+        if (N % p != 0) return -1;
+        const int64_t Np = N / p;
+        double* Pi = (double*)malloc((size_t)(T * K) * sizeof(double));
+        double* dWi = (double*)malloc((size_t)(K * Np) * sizeof(double));
+        memset(dX, 0, (size_t)(T * K) * sizeof(double));
+        for (int i = 0; i < p; ++i) {
+            double* Wi = col_block(K, N, W, i * Np, Np);
+            double* dYi = col_block(T, N, dY, i * Np, Np);
+            mm_tn(K, Np, T, X, dYi, dWi);
+            for (int64_t k = 0; k < K; ++k)
+                memcpy(dW + k * N + i * Np, dWi + k * Np, (size_t)Np * sizeof(double));
+            mm_nt(T, K, Np, dYi, Wi, Pi);
+            for (int64_t e = 0; e < T * K; ++e) dX[e] += Pi[e];
+            free(Wi);
+            free(dYi);
+        }
+        free(Pi);
+        free(dWi);
+        return 0;
+    }
+    if (K % p != 0) return -1;
+    const int64_t Kp = K / p;
+    double* dXi = (double*)malloc((size_t)(T * Kp) * sizeof(double));
+    for (int i = 0; i < p; ++i) {
+        const double* Wi = W + (int64_t)i * Kp * N;
+        double* Xi = col_block(T, K, X, i * Kp, Kp);
+        mm_nt(T, Kp, N, dY, Wi, dXi);
+        for (int64_t t = 0; t < T; ++t)
+            memcpy(dX + t * K + i * Kp, dXi + t * Kp, (size_t)Kp * sizeof(double));
+        mm_tn(Kp, N, T, Xi, dY, dW + (int64_t)i * Kp * N);
+        free(Xi);
+    }
+    free(dXi);
+    return 0;
+}

@@ -349,6 +349,103 @@ def test_torch_float64_autograd(act):
         assert _max_rel(got[k], v.detach().numpy()) < 1e-12, k
 
 
+# ------------------------------------------- tensor-parallel linear layers
+
+def _rand_linear(rng, T, K, N):
+    return dict(X=rng.standard_normal((T, K)), W=rng.standard_normal((K, N)) * 0.7,
+                bias=rng.standard_normal(N) * 0.5, dY=rng.standard_normal((T, N)))
+
+
+def check_linear_bruteforce(orc, seed=8):
+    rng = np.random.default_rng(seed)
+    for T, K, N in [(1, 1, 1), (3, 4, 6), (5, 6, 4), (7, 8, 12)]:
+        P = _rand_linear(rng, T, K, N)
+        Y = orc.linear_forward(P["X"], P["W"], P["bias"])
+        dX, dW, db = orc.linear_backward(P["X"], P["W"], P["dY"])
+        ref = bruteforce.linear(*(P[k].tolist() for k in ("X", "W", "bias", "dY")))
+        for k, v in dict(Y=Y, dX=dX, dW=dW, db=db).items():
+            assert _max_rel(v, ref[k]) <= 1e-12, (k, T, K, N)
+
+
+def test_linear_bruteforce():
+    check_linear_bruteforce(oracle.default())
+
+
+def test_linear_finite_differences():
+    """L = Σ dY ⊙ Y; central differences pin dX, dW, dbias."""
+    rng = np.random.default_rng(9)
+    P = _rand_linear(rng, 4, 5, 6)
+    dX, dW, db = oracle.linear_backward(P["X"], P["W"], P["dY"])
+
+    def loss(Q):
+        return float(np.sum(P["dY"] * oracle.linear_forward(Q["X"], Q["W"], Q["bias"])))
+
+    for name, g in (("X", dX), ("W", dW), ("bias", db)):
+        for idx in rng.choice(P[name].size, size=5, replace=False):
+            Qp = {k: v.copy() for k, v in P.items()}
+            Qm = {k: v.copy() for k, v in P.items()}
+            Qp[name].reshape(-1)[idx] += 1e-6
+            Qm[name].reshape(-1)[idx] -= 1e-6
+            fd = (loss(Qp) - loss(Qm)) / 2e-6
+            assert abs(fd - g.reshape(-1)[idx]) <= 1e-7 * max(1.0, abs(fd)), (name, idx)
+
+
+@pytest.mark.parametrize("split", ["columns", "rows"])
+def test_linear_partition_identities(split):
+    """Column split: concatenated X·W_i + bias_i equals X·W + bias bit for bit;
+    row split: Σ_i X_i·W_i + bias equals it within rounding; both backward
+    partitions give the unsplit gradients."""
+    rng = np.random.default_rng(10)
+    T, K, N = 6, 12, 24
+    P = _rand_linear(rng, T, K, N)
+    Y = oracle.linear_forward(P["X"], P["W"], P["bias"])
+    dX, dW, db = oracle.linear_backward(P["X"], P["W"], P["dY"])
+    dim = N if split == "columns" else K
+    for p in [d for d in range(1, dim + 1) if dim % d == 0]:
+        Ys = oracle.linear_forward_sharded(P["X"], P["W"], P["bias"], p, split)
+        if split == "columns":
+            np.testing.assert_array_equal(Ys, Y)
+        else:
+            assert _max_rel(Ys, Y) < 1e-13, p
+        gs = oracle.linear_backward_sharded(P["X"], P["W"], P["dY"], p, split)
+        for a, b in zip(gs, (dX, dW, db)):
+            assert _max_rel(a, b) < 1e-13, (split, p)
+    with pytest.raises(ValueError):
+        oracle.linear_forward_sharded(P["X"], P["W"], P["bias"], 5, split)
+
+
+def test_mlp_is_column_linear_gelu_row_linear():
+    """The block composes the two layers: H = column-linear(X; A, a),
+    Z = row-linear(GeLU(H); B, b), and the backward chains through GeLU′."""
+    rng = np.random.default_rng(11)
+    P = _rand_problem(rng, 5, 6, 12)
+    full = _all_outputs(oracle.default(), P)
+    H = oracle.linear_forward(P["X"], P["A"], P["a"])
+    np.testing.assert_allclose(H, full["H"], rtol=0, atol=1e-14)
+    Z = oracle.linear_forward(full["Y"], P["B"], P["b"])
+    np.testing.assert_allclose(Z, full["Z"], rtol=0, atol=1e-13)
+    dY, dB, db = oracle.linear_backward(full["Y"], P["B"], P["dZ"])
+    np.testing.assert_allclose(dB, full["dB"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(db, full["db"], rtol=0, atol=1e-13)
+    dX, dA, da = oracle.linear_backward(P["X"], P["A"], full["dH"])
+    np.testing.assert_allclose(dX, full["dX"], rtol=0, atol=1e-13)
+    np.testing.assert_allclose(dA, full["dA"], rtol=0, atol=1e-13)
+
+
+def test_linear_torch_float64_autograd():
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(12)
+    P = _rand_linear(rng, 9, 7, 11)
+    t = {k: torch.tensor(v, dtype=torch.float64, requires_grad=k != "dY") for k, v in P.items()}
+    Y = t["X"] @ t["W"] + t["bias"]
+    (Y * t["dY"]).sum().backward()
+    got = oracle.linear_forward(P["X"], P["W"], P["bias"])
+    dX, dW, db = oracle.linear_backward(P["X"], P["W"], P["dY"])
+    assert _max_rel(got, Y.detach().numpy()) < 1e-13
+    for a, b in ((dX, t["X"].grad), (dW, t["W"].grad), (db, t["bias"].grad)):
+        assert _max_rel(a, b.numpy()) < 1e-13
+
+
 # ------------------------------------------------------- planted mistakes
 
 MUTANTS = {
@@ -365,6 +462,9 @@ MUTANTS = {
     "dropped_bias": ("H[t * F + f] += a[f];", "H[t * F + f] += 0.0 * a[f];"),
     # wrong cubic coefficient in the tanh form
     "wrong_tanh_constant": ("#define TPO_GELU_TANH_C 0.044715", "#define TPO_GELU_TANH_C 0.04"),
+    # linear-layer bias added twice
+    "linear_bias_twice": ("for (int64_t n = 0; n < N; ++n) Y[t * N + n] += bias[n];",
+                          "for (int64_t n = 0; n < N; ++n) Y[t * N + n] += 2.0 * bias[n];"),
     # db summing the wrong tensor's columns
     "wrong_index": ("tpo_colsum(T, h, dZ, db);\n    mm_tn(F, h, T, Y, dZ, dB);",
                     "tpo_colsum(T, h, dZ, db);\n    mm_tn(F, h, T, H, dZ, dB);"),
@@ -372,7 +472,8 @@ MUTANTS = {
 
 
 def _catches(orc):
-    checks = [check_hand_example, check_bruteforce, check_finite_differences, check_normal_table]
+    checks = [check_hand_example, check_bruteforce, check_finite_differences, check_normal_table,
+              check_linear_bruteforce]
     for chk in checks:
         for act in (0, 1):
             try:
