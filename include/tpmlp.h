@@ -113,6 +113,33 @@ tpmlp_status tp_mlp_bwd_ex(const void* dZ, const void* X, const void* A, const v
                            tpmlp_dtype dt, tpmlp_activation act, void* workspace,
                            size_t workspace_bytes, void* stream);
 
+/* Tensor-parallel linear layer Y = X·W + bias, X: T×K, W: K×N, bias: N (may
+ * be NULL), all of dtype dt; the attention layer's use of the two splits
+ * (page "Megatron", section "Transformer层的张量并行实现": the QKV projection is
+ * split by columns, the output projection by rows; section "张量并行 /
+ * 数学原理" for the splits themselves).
+ *   TPMLP_SPLIT_COLUMNS: W = [W_1 … W_p] (N % p == 0). Forward Y_i = X·W_i +
+ *     bias_i side by side, no exchange. Backward dW_i = Xᵀ·dY_i, dbias_i =
+ *     1ᵀ·dY_i and, X being replicated, dX = Σ_{i=1..p} dY_i·W_iᵀ summed in
+ *     ascending i.
+ *   TPMLP_SPLIT_ROWS: W = [W_1; …; W_p] (K % p == 0), X split into the
+ *     matching column blocks X_i. Forward Y = Σ_{i=1..p} X_i·W_i + bias,
+ *     ascending i, bias once. Backward dX_i = dY·W_iᵀ (no exchange), dW_i =
+ *     X_iᵀ·dY, dbias = 1ᵀ·dY.
+ * dW (K×N) and dbias (N) are fp32; dX (T×K) and Y (T×N) have dtype dt.
+ * Requirements, alignment and error behaviour as tp_mlp_fwd, with K and N in
+ * place of h and F. With T == 0, dW and dbias are set to zero. */
+typedef enum tpmlp_split { TPMLP_SPLIT_COLUMNS = 0, TPMLP_SPLIT_ROWS = 1 } tpmlp_split;
+
+size_t tpmlp_linear_workspace_size(int64_t T, int64_t K, int64_t N, int p, tpmlp_split split,
+                                   tpmlp_dtype dt);
+tpmlp_status tp_linear_fwd(const void* X, const void* W, const void* bias, void* Y, int64_t T,
+                           int64_t K, int64_t N, int p, tpmlp_split split, tpmlp_dtype dt,
+                           void* workspace, size_t workspace_bytes, void* stream);
+tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* dX, float* dW,
+                           float* dbias, int64_t T, int64_t K, int64_t N, int p, tpmlp_split split,
+                           tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* tpmlp_strerror(tpmlp_status s);
 

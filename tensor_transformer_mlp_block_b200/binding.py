@@ -22,7 +22,7 @@ ACTIVATIONS = {"gelu": 0, "gelu_tanh": 1}
 # The entry points include/tpmlp.h declares, in declaration order.
 EXPORTS = (
     "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tp_mlp_fwd_ex", "tp_mlp_bwd_ex",
-    "tpmlp_strerror",
+    "tpmlp_linear_workspace_size", "tp_linear_fwd", "tp_linear_bwd", "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
@@ -63,6 +63,15 @@ def lib() -> ctypes.CDLL:
             L.tp_mlp_bwd_ex.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
                                                     ctypes.c_int, vp, sz, vp]
             L.tp_mlp_bwd_ex.restype = ctypes.c_int
+            L.tpmlp_linear_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                      ctypes.c_int]
+            L.tpmlp_linear_workspace_size.restype = sz
+            L.tp_linear_fwd.argtypes = [vp] * 4 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, vp, sz, vp]
+            L.tp_linear_fwd.restype = ctypes.c_int
+            L.tp_linear_bwd.argtypes = [vp] * 6 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
+                                                   ctypes.c_int, vp, sz, vp]
+            L.tp_linear_bwd.restype = ctypes.c_int
             L.tpmlp_strerror.argtypes = [ctypes.c_int]
             L.tpmlp_strerror.restype = ctypes.c_char_p
             L.tpmlp_last_device_status.argtypes = [vp]
@@ -293,3 +302,64 @@ def eval_activation(x: torch.Tensor, form: int):
                                        int(form), _stream_ptr(x.device, None)),
            "tpmlp_eval_activation")
     return y, dy
+
+
+SPLITS = {"columns": 0, "rows": 1}
+
+
+def _split_code(split: str) -> int:
+    try:
+        return SPLITS[split]
+    except KeyError:
+        raise ValueError(f"split must be one of {sorted(SPLITS)}") from None
+
+
+def linear_workspace_size(T: int, K: int, N: int, p: int, split: str,
+                          dtype: torch.dtype = torch.bfloat16) -> int:
+    code = BF16 if dtype == torch.bfloat16 else FP32
+    return int(lib().tpmlp_linear_workspace_size(T, K, N, p, _split_code(split), code))
+
+
+def linear_forward(X, W, bias, p: int, split: str, *, out=None, workspace=None, stream=None):
+    """Y = X·W + bias with W split into p shards by "columns" (QKV-style) or
+    "rows" (output-projection style). X: T×K, W: K×N, bias: N or None."""
+    T, K = X.shape
+    N = W.shape[1]
+    dt, dev = X.dtype, X.device
+    _need(X, "X", (T, K), dt, dev)
+    _need(W, "W", (K, N), dt, dev)
+    if bias is not None:
+        _need(bias, "bias", (N,), dt, dev)
+    Y = torch.empty((T, N), dtype=dt, device=dev) if out is None else out
+    _need(Y, "Y", (T, N), dt, dev)
+    n = linear_workspace_size(T, K, N, p, split, dt)
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
+    st = lib().tp_linear_fwd(_ptr(X), _ptr(W), _ptr(bias), _ptr(Y), T, K, N, int(p),
+                             _split_code(split), _dtype_code(X), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
+    _check(st, "tp_linear_fwd")
+    return Y
+
+
+def linear_backward(dY, X, W, p: int, split: str, *, out=None, workspace=None, stream=None):
+    """(dX, dW, dbias) of linear_forward for upstream dY (T×N); dW and dbias fp32."""
+    T, K = X.shape
+    N = W.shape[1]
+    dt, dev = X.dtype, X.device
+    for name, t, shp in (("dY", dY, (T, N)), ("X", X, (T, K)), ("W", W, (K, N))):
+        _need(t, name, shp, dt, dev)
+    if out is None:
+        out = (torch.empty((T, K), dtype=dt, device=dev),
+               torch.empty((K, N), dtype=torch.float32, device=dev),
+               torch.empty((N,), dtype=torch.float32, device=dev))
+    dX, dW, db = out
+    _need(dX, "dX", (T, K), dt, dev)
+    _need(dW, "dW", (K, N), torch.float32, dev)
+    _need(db, "dbias", (N,), torch.float32, dev)
+    n = linear_workspace_size(T, K, N, p, split, dt)
+    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
+    st = lib().tp_linear_bwd(_ptr(dY), _ptr(X), _ptr(W), _ptr(dX), _ptr(dW), _ptr(db), T, K, N,
+                             int(p), _split_code(split), _dtype_code(X), _ptr(ws),
+                             ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
+    _check(st, "tp_linear_bwd")
+    return dX, dW, db

@@ -16,6 +16,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cstdint>
 #include <cstring>
@@ -139,12 +140,15 @@ tpmlp_status check_launch() {
 // ------------------------------------------------------- per-kernel timing
 
 enum Kind : int {
-    K_F1 = 0, K_F2, K_F2_RED, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_B5_RED, K_MISC, K_COUNT
+    K_F1 = 0, K_F2, K_F2_RED, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_B5_RED, K_MISC,
+    K_L_FWD, K_L_FWD_RED, K_L_DB, K_L_DW, K_L_DX, K_L_DX_RED, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "F2.split_reduce", "B1.db_colsum",
     "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
     "B5.dgrad_dX_shard_sum", "B5.split_reduce",       "misc",
+    "L.fwd_gemm_bias",       "L.fwd_split_reduce",    "L.dbias_colsum",  "L.wgrad_dW",
+    "L.dgrad_dX",            "L.dgrad_split_reduce",
 };
 
 struct KindTotals {
@@ -489,6 +493,151 @@ tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype d
     return TPMLP_OK;
 }
 
+// ------------------------------------------------ tensor-parallel linear
+
+// Plan of a linear layer Y = X·W + bias (X: T × K, W: K × N), W split into
+// p shards by columns (split 0) or rows (split 1). The product carrying a
+// shard sum (the forward for rows, dX of the backward for columns) may be
+// split by shard like the MLP's row-parallel products.
+struct LinPlan {
+    bool tc = false;
+    int splits_fwd = 1, splits_bwd = 1;
+    int64_t chunks = 1;
+    size_t off_split = 0, off_cs = 0, total = 0;
+};
+
+bool make_lin_plan(int64_t T, int64_t K, int64_t N, int p, int split, tpmlp_dtype dt, LinPlan* pl) {
+    if (T < 0 || K < 1 || N < 1 || p < 1 || (split != 0 && split != 1)) return false;
+    if (split == 0 && N % p != 0) return false;
+    if (split == 1 && K % p != 0) return false;
+    if (dt != TPMLP_BF16 && dt != TPMLP_FP32) return false;
+    pl->tc = (dt == TPMLP_BF16) && (K % 8 == 0) && (N % 8 == 0);
+    int num_sms = 148;
+    if (const DeviceInfo* d = device_info()) num_sms = d->num_sms;
+    if (pl->tc) {
+        if (split == 1) pl->splits_fwd = choose_splits(T, N, K, p, num_sms);
+        else pl->splits_bwd = choose_splits(T, K, N, p, num_sms);
+    }
+    pl->chunks = T > 0 ? (T + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk : 1;
+    size_t split_bytes = 0;
+    if (pl->splits_fwd > 1) split_bytes = static_cast<size_t>(pl->splits_fwd) * T * N * sizeof(float);
+    if (pl->splits_bwd > 1)
+        split_bytes = std::max(split_bytes, static_cast<size_t>(pl->splits_bwd) * T * K * sizeof(float));
+    pl->off_split = 0;
+    pl->off_cs = round256(split_bytes);
+    pl->total = pl->off_cs + round256(static_cast<size_t>(pl->chunks) * N * sizeof(float));
+    return true;
+}
+
+tpmlp_status lin_checks(int64_t T, int64_t K, int64_t N, int p, int split, tpmlp_dtype dt,
+                        LinPlan* pl, void* ws, size_t ws_bytes) {
+    if (!make_lin_plan(T, K, N, p, split, dt, pl)) return TPMLP_ERR_INVALID;
+    if (T >= (int64_t(1) << 31) || K >= (int64_t(1) << 31) || N >= (int64_t(1) << 31))
+        return TPMLP_ERR_UNSUPPORTED;
+    const DeviceInfo* d = device_info();
+    if (d == nullptr) return TPMLP_ERR_CUDA;
+    if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
+    if (pl->total > 0 && (ws == nullptr || ws_bytes < pl->total)) return TPMLP_ERR_WORKSPACE;
+    if (ws != nullptr && !aligned16(ws)) return TPMLP_ERR_ALIGN;
+    return TPMLP_OK;
+}
+
+tpmlp_status linear_fwd_impl(const void* X, const void* W, const void* bias, void* Y, int64_t T,
+                             int64_t K, int64_t N, int p, int split, tpmlp_dtype dt, void* workspace,
+                             size_t workspace_bytes, cudaStream_t st) {
+    LinPlan pl;
+    TPMLP_TRY(lin_checks(T, K, N, p, split, dt, &pl, workspace, workspace_bytes));
+    if (T == 0) return TPMLP_OK;
+    if (!X || !W || !Y) return TPMLP_ERR_INVALID;
+    const int iT = static_cast<int>(T), iK = static_cast<int>(K), iN = static_cast<int>(N);
+    if (pl.tc) {
+        for (const void* q : {X, W, bias, static_cast<const void*>(Y)})
+            if (q && !aligned16(q)) return TPMLP_ERR_ALIGN;
+        // Aop = X [T][K] (K-major), Bop = W [K][N] (MN-major)
+        GemmArgs g{};
+        if (pl.splits_fwd == 1) {
+            g.out0 = Y;
+            g.ld_out = N;
+            g.bias = static_cast<const __nv_bfloat16*>(bias);
+            return gemm_tc<256, false, true, EPI_BIAS>(K_L_FWD, X, W, iT, iN, iK, 1, g, st);
+        }
+        float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
+        g.out0 = ws;
+        g.ld_out = N;
+        g.split_stride = T * N;
+        TPMLP_TRY((gemm_tc<256, false, true, EPI_F32>(K_L_FWD, X, W, iT, iN, iK, pl.splits_fwd, g, st)));
+        return reduce_splits(K_L_FWD_RED, ws, pl.splits_fwd, T, N, bias, Y, st);
+    }
+    SimtArgs a{};
+    a.M = iT; a.N = iN; a.K = iK;
+    a.A = X; a.sam = K; a.sak = 1;
+    a.B = W; a.sbk = N; a.sbn = 1;
+    a.out0 = Y; a.ld_out = N; a.bias = bias;
+    if (dt == TPMLP_FP32) return gemm_simt<float, EPI_BIAS>(K_L_FWD, a, st);
+    return gemm_simt<__nv_bfloat16, EPI_BIAS>(K_L_FWD, a, st);
+}
+
+tpmlp_status linear_bwd_impl(const void* dY, const void* X, const void* W, void* dX, float* dW,
+                             float* dbias, int64_t T, int64_t K, int64_t N, int p, int split,
+                             tpmlp_dtype dt, void* workspace, size_t workspace_bytes,
+                             cudaStream_t st) {
+    LinPlan pl;
+    TPMLP_TRY(lin_checks(T, K, N, p, split, dt, &pl, workspace, workspace_bytes));
+    if (!dW || !dbias) return TPMLP_ERR_INVALID;
+    if (T == 0) {
+        TPMLP_TRY(zero_f32(dW, K * N, st));
+        return zero_f32(dbias, N, st);
+    }
+    if (!dY || !X || !W || !dX) return TPMLP_ERR_INVALID;
+    float* cs = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_cs);
+    const int iT = static_cast<int>(T), iK = static_cast<int>(K), iN = static_cast<int>(N);
+    if (pl.tc) {
+        for (const void* q : {dY, X, W, static_cast<const void*>(dX), static_cast<const void*>(dW),
+                              static_cast<const void*>(dbias)})
+            if (!aligned16(q)) return TPMLP_ERR_ALIGN;
+        TPMLP_TRY(colsum(K_L_DB, static_cast<const __nv_bfloat16*>(dY), T, N, pl.chunks, cs, dbias, st));
+        // dW = Xᵀ·dY: Aop = X [T][K] (MN-major, M = K), Bop = dY [T][N] (MN-major)
+        GemmArgs gw{};
+        gw.out0 = dW;
+        gw.ld_out = N;
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_L_DW, X, dY, iK, iN, iT, 1, gw, st)));
+        // dX = dY·Wᵀ: Aop = dY [T][N] (K-major), Bop = W [K][N] read as [N' = K][K' = N] (K-major);
+        // for the column split this is the shard sum over the N dimension
+        GemmArgs gx{};
+        if (pl.splits_bwd == 1) {
+            gx.out0 = dX;
+            gx.ld_out = K;
+            return gemm_tc<256, false, false, EPI_BIAS>(K_L_DX, dY, W, iT, iK, iN, 1, gx, st);
+        }
+        float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
+        gx.out0 = ws;
+        gx.ld_out = K;
+        gx.split_stride = T * K;
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_F32>(K_L_DX, dY, W, iT, iK, iN, pl.splits_bwd, gx, st)));
+        return reduce_splits(K_L_DX_RED, ws, pl.splits_bwd, T, K, nullptr, dX, st);
+    }
+    // dW = Xᵀ·dY: Aop(k, t) = X[t][k], Bop(t, n) = dY[t][n]
+    SimtArgs w{};
+    w.M = iK; w.N = iN; w.K = iT;
+    w.A = X; w.sam = 1; w.sak = K;
+    w.B = dY; w.sbk = N; w.sbn = 1;
+    w.out0 = dW; w.ld_out = N;
+    // dX = dY·Wᵀ: Aop(t, n) = dY[t][n], Bop(n, k) = W[k][n]
+    SimtArgs x{};
+    x.M = iT; x.N = iK; x.K = iN;
+    x.A = dY; x.sam = N; x.sak = 1;
+    x.B = W; x.sbk = 1; x.sbn = N;
+    x.out0 = dX; x.ld_out = K;
+    if (dt == TPMLP_FP32) {
+        TPMLP_TRY(colsum(K_L_DB, static_cast<const float*>(dY), T, N, pl.chunks, cs, dbias, st));
+        TPMLP_TRY((gemm_simt<float, EPI_F32>(K_L_DW, w, st)));
+        return gemm_simt<float, EPI_BIAS>(K_L_DX, x, st);
+    }
+    TPMLP_TRY(colsum(K_L_DB, static_cast<const __nv_bfloat16*>(dY), T, N, pl.chunks, cs, dbias, st));
+    TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_F32>(K_L_DW, w, st)));
+    return gemm_simt<__nv_bfloat16, EPI_BIAS>(K_L_DX, x, st);
+}
+
 // Forward with activation epilogue EPI_ACT (EPI_GELU or EPI_GELU_TANH).
 template <int EPI_ACT>
 tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B, const void* b,
@@ -715,6 +864,29 @@ tpmlp_status tp_mlp_bwd_ex(const void* dZ, const void* X, const void* A, const v
                                             dt, workspace, workspace_bytes, stream);
     }
     return TPMLP_ERR_INVALID;
+}
+
+size_t tpmlp_linear_workspace_size(int64_t T, int64_t K, int64_t N, int p, tpmlp_split split,
+                                   tpmlp_dtype dt) {
+    LinPlan pl;
+    if (!make_lin_plan(T, K, N, p, static_cast<int>(split), dt, &pl)) return 0;
+    return pl.total;
+}
+
+tpmlp_status tp_linear_fwd(const void* X, const void* W, const void* bias, void* Y, int64_t T,
+                           int64_t K, int64_t N, int p, tpmlp_split split, tpmlp_dtype dt,
+                           void* workspace, size_t workspace_bytes, void* stream) {
+    cudaGetLastError();
+    return linear_fwd_impl(X, W, bias, Y, T, K, N, p, static_cast<int>(split), dt, workspace,
+                           workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* dX, float* dW,
+                           float* dbias, int64_t T, int64_t K, int64_t N, int p, tpmlp_split split,
+                           tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+    cudaGetLastError();
+    return linear_bwd_impl(dY, X, W, dX, dW, dbias, T, K, N, p, static_cast<int>(split), dt,
+                           workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
 const char* tpmlp_strerror(tpmlp_status s) {
