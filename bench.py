@@ -49,6 +49,11 @@ def parse_args(argv=None):
     ap.add_argument("--e2e-steps", type=int, default=30)
     ap.add_argument("--graph", action="store_true",
                     help="capture one step in a CUDA graph and time its replays")
+    ap.add_argument("--activation", choices=["gelu", "gelu_tanh"], default="gelu",
+                    help="MLP activation: exact GeLU (default) or its tanh approximation")
+    ap.add_argument("--block", choices=["mlp", "attn-proj"], default="mlp",
+                    help="mlp: the MLP block (default); attn-proj: the attention layer's "
+                         "tensor-parallel projections (QKV split by columns, output by rows)")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (for profiler runs)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -275,13 +280,49 @@ def bench_ours(args, cfg, world, rank, local):
     ws = torch.empty(max(binding.workspace_size(T, h, F, p, dt), 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    act = args.activation
+
     def step(x=None, dz=None):
         x = d["X"] if x is None else x
         dz = d["dZ"] if dz is None else dz
-        binding.forward(x, d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, Z), workspace=ws)
-        binding.backward(dz, x, d["A"], d["B"], H, Y, p, out=gout, workspace=ws)
+        binding.forward(x, d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, Z), workspace=ws,
+                        activation=act)
+        binding.backward(dz, x, d["A"], d["B"], H, Y, p, out=gout, workspace=ws, activation=act)
 
     working_set = sum(t.numel() * t.element_size() for t in [*d.values(), H, Y, Z, *gout.values()])
+    flops_per_step = cfg.flops_fwd_bwd
+    if args.block == "attn-proj":
+        # the attention layer's two tensor-parallel projections at this width:
+        # QKV = X·W_qkv (h -> 3h, columns), Z = O·W_o (h -> h, rows), fwd + bwd
+        del H, Y, gout
+        torch.cuda.empty_cache()
+        gen = torch.Generator().manual_seed(21)
+        Wqkv = (torch.randn((h, 3 * h), generator=gen) * 0.02).to(dt).to(dev)
+        bqkv = torch.zeros((3 * h,), dtype=dt, device=dev)
+        Wo = (torch.randn((h, h), generator=gen) * 0.02).to(dt).to(dev)
+        bo = torch.zeros((h,), dtype=dt, device=dev)
+        O = torch.randn((T, h), generator=gen).to(dt).to(dev)
+        dQKV = torch.randn((T, 3 * h), generator=gen).to(dt).to(dev)
+        QKV = torch.empty((T, 3 * h), dtype=dt, device=dev)
+        g_qkv = (torch.empty((T, h), dtype=dt, device=dev), torch.empty((h, 3 * h), dtype=f32, device=dev),
+                 torch.empty((3 * h,), dtype=f32, device=dev))
+        g_o = (torch.empty((T, h), dtype=dt, device=dev), torch.empty((h, h), dtype=f32, device=dev),
+               torch.empty((h,), dtype=f32, device=dev))
+        ws_l = torch.empty(max(binding.linear_workspace_size(T, h, 3 * h, p, "columns", dt),
+                               binding.linear_workspace_size(T, h, h, p, "rows", dt), 1),
+                           dtype=torch.uint8, device=dev)
+
+        def step(x=None, dz=None):
+            x = d["X"] if x is None else x
+            dz = d["dZ"] if dz is None else dz
+            binding.linear_forward(x, Wqkv, bqkv, p, "columns", out=QKV, workspace=ws_l)
+            binding.linear_backward(dQKV, x, Wqkv, p, "columns", out=g_qkv, workspace=ws_l)
+            binding.linear_forward(O, Wo, bo, p, "rows", out=Z, workspace=ws_l)
+            binding.linear_backward(dz, O, Wo, p, "rows", out=g_o, workspace=ws_l)
+
+        flops_per_step = 24.0 * T * h * h
+        working_set = sum(t.numel() * t.element_size()
+                          for t in [d["X"], d["dZ"], Wqkv, Wo, O, dQKV, QKV, Z, *g_qkv, *g_o])
 
     for _ in range(args.warmup):
         step()
@@ -343,7 +384,7 @@ def bench_ours(args, cfg, world, rank, local):
         raise RuntimeError(f"device status {status} after the timed region")
     seconds = e0.elapsed_time(e1) / 1e3
     max_seconds = max_over_ranks(seconds, dev)
-    agg = aggregate(cfg.flops_fwd_bwd, args.steps, max_seconds, world)
+    agg = aggregate(flops_per_step, args.steps, max_seconds, world)
 
     # dominant kernel and its roofline (tensor-bound: algorithmic flops / event time)
     top_name, top = max(kinds.items(), key=lambda kv: kv[1]["ms"])
@@ -361,6 +402,23 @@ def bench_ours(args, cfg, world, rank, local):
                       "gbs": v["bytes"] / v["ms"] / 1e6}
                   for k, v in kinds.items()}
 
+    if args.block != "mlp":
+        e2e = None
+    else:
+        e2e = e2e_measure(args, cfg, inp, d, H, Y, Z, gout, ws, p, T, h, dt, dev, stream, world, act,
+                          binding, torch)
+
+    line = _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, launches,
+                 clocks, working_set, flops_per_step, T, h, F, p)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.block == "mlp":
+        line["cpu_baseline"] = cpu_baseline(inp, cfg, args.cpu_seconds)
+    elif rank == 0:
+        line["cpu_baseline"] = None
+    return line
+
+
+def e2e_measure(args, cfg, inp, d, H, Y, Z, gout, ws, p, T, h, dt, dev, stream, world, act,
+                binding, torch):
     # End to end through the public API with pinned host buffers: every step
     # copies its X and dZ in from pinned host memory and its Z and dX back
     # out. The copies run on two copy streams, double-buffered, so step i's
@@ -399,9 +457,10 @@ def bench_ours(args, cfg, world, rank, local):
             if i >= 2:
                 stream.wait_event(ev_out[b])  # step i-2's outputs are on the host
             binding.forward(xin[b], d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, zout[b]),
-                            workspace=ws)
+                            workspace=ws, activation=act)
             gout["dX"] = dxout[b]
-            binding.backward(dzin[b], xin[b], d["A"], d["B"], H, Y, p, out=gout, workspace=ws)
+            binding.backward(dzin[b], xin[b], d["A"], d["B"], H, Y, p, out=gout, workspace=ws,
+                             activation=act)
             ev_comp[b].record(stream)
             with torch.cuda.stream(s_out):
                 s_out.wait_event(ev_comp[b])
@@ -421,15 +480,31 @@ def bench_ours(args, cfg, world, rank, local):
     assert torch.equal(hZ, zout[(args.e2e_steps - 1) % 2].cpu())
     bytes_in = hX.numel() * hX.element_size() + hdZ.numel() * hdZ.element_size()
     bytes_out = hZ.numel() * hZ.element_size() + hdX.numel() * hdX.element_size()
+    return {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": bytes_in,
+            "d2h_bytes_per_step": bytes_out, "steps": args.e2e_steps,
+            "what": "per step: X and dZ copied in from pinned host memory, fwd+bwd through the "
+                    "public API, Z and dX copied out to pinned host memory; copies pipelined on "
+                    "two copy streams with double-buffered device tensors; weights and weight "
+                    "gradients stay resident"}
 
-    line = {
-        "metric": METRIC, "value": agg["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
+
+def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, launches, clocks,
+          working_set, flops_per_step, T, h, F, p):
+    workload = f"{cfg.name}-class TP-MLP fwd+bwd"
+    if args.block == "attn-proj":
+        workload = f"{cfg.name}-class attention projections (QKV columns + output rows) fwd+bwd"
+    elif args.activation != "gelu":
+        workload += f" ({args.activation})"
+    metric = METRIC if args.block == "mlp" else \
+        "TP attention projections fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
+    return {
+        "metric": metric, "value": agg["value"], "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": agg["ms_per_step"], "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if cfg.dtype == "bf16" else "fp32",
         "data": "synthetic (seeded Gaussian inputs, random-init weights of the named shapes)",
-        "config": {"workload": f"{cfg.name}-class TP-MLP fwd+bwd", "T": T, "h": h, "F": F, "p": p,
-                   "flops_per_step": cfg.flops_fwd_bwd, "parallelism": f"replicas x{world}",
-                   "cuda_graph": bool(args.graph),
+        "config": {"workload": workload, "T": T, "h": h, "F": F, "p": p,
+                   "flops_per_step": flops_per_step, "parallelism": f"replicas x{world}",
+                   "cuda_graph": bool(args.graph), "activation": args.activation,
                    "l2": f"working set {working_set / 2**30:.2f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB "
                          "(inputs larger than L2; no flush)"},
         "frac_of_peak": {"measured_burst": agg["value"] / world / peaks["bf16_tflops"],
@@ -438,20 +513,10 @@ def bench_ours(args, cfg, world, rank, local):
                          "peaks": peaks_src},
         "roofline": roofline,
         "kernels": per_kernel,
-        "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": bytes_in,
-                "d2h_bytes_per_step": bytes_out, "steps": args.e2e_steps,
-                "what": "per step: X and dZ copied in from pinned host memory, fwd+bwd through the "
-                        "public API, Z and dX copied out to pinned host memory; copies pipelined on "
-                        "two copy streams with double-buffered device tensors; weights and weight "
-                        "gradients stay resident"},
+        "e2e": e2e,
         "gpu_launches": launches,
         "clocks": clocks,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inp, cfg, args.cpu_seconds)
-    elif rank == 0:
-        line["cpu_baseline"] = None
-    return line
 
 
 # ---------------------------------------------------------- reference arm
