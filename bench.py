@@ -51,6 +51,8 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--activation", choices=["gelu", "gelu_tanh"], default="gelu",
                     help="MLP activation: exact GeLU (default) or its tanh approximation")
+    ap.add_argument("--recompute", action="store_true",
+                    help="activation recompute: rebuild Y from H before each backward")
     ap.add_argument("--block", choices=["mlp", "attn-proj"], default="mlp",
                     help="mlp: the MLP block (default); attn-proj: the attention layer's "
                          "tensor-parallel projections (QKV split by columns, output by rows)")
@@ -287,6 +289,8 @@ def bench_ours(args, cfg, world, rank, local):
         dz = d["dZ"] if dz is None else dz
         binding.forward(x, d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, Z), workspace=ws,
                         activation=act)
+        if args.recompute:
+            binding.recompute_activation(H, out=Y, activation=act)
         binding.backward(dz, x, d["A"], d["B"], H, Y, p, out=gout, workspace=ws, activation=act)
 
     working_set = sum(t.numel() * t.element_size() for t in [*d.values(), H, Y, Z, *gout.values()])
@@ -493,8 +497,11 @@ def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, la
     workload = f"{cfg.name}-class TP-MLP fwd+bwd"
     if args.block == "attn-proj":
         workload = f"{cfg.name}-class attention projections (QKV columns + output rows) fwd+bwd"
-    elif args.activation != "gelu":
-        workload += f" ({args.activation})"
+    else:
+        if args.activation != "gelu":
+            workload += f" ({args.activation})"
+        if args.recompute:
+            workload += " with activation recompute"
     metric = METRIC if args.block == "mlp" else \
         "TP attention projections fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
     return {

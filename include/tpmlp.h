@@ -140,6 +140,19 @@ tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* d
                            float* dbias, int64_t T, int64_t K, int64_t N, int p, tpmlp_split split,
                            tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream);
 
+/* Activation recompute (page "Megatron", section "其他关键技术 / 激活重计算":
+ * keep fewer forward activations and recompute them in the backward). A
+ * caller that keeps only the pre-activation H after tp_mlp_fwd(_ex) rebuilds
+ * Y = act(H) here just before tp_mlp_bwd(_ex):
+ *   Y[i] = act(H[i]), i < n (n = T·F), H and Y device arrays of dtype dt,
+ *   act = the forward's activation.
+ * One bandwidth-bound pass (n reads, n writes). Y rebuilt from the stored H
+ * (rounded to dt) can differ from the forward's Y (computed from the fp32
+ * accumulator) by the effect of that one rounding. Returns
+ * TPMLP_ERR_INVALID for n < 0, null pointers, or an unknown dt or act. */
+tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpmlp_dtype dt,
+                                         tpmlp_activation act, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* tpmlp_strerror(tpmlp_status s);
 

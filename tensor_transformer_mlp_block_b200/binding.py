@@ -22,7 +22,8 @@ ACTIVATIONS = {"gelu": 0, "gelu_tanh": 1}
 # The entry points include/tpmlp.h declares, in declaration order.
 EXPORTS = (
     "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tp_mlp_fwd_ex", "tp_mlp_bwd_ex",
-    "tpmlp_linear_workspace_size", "tp_linear_fwd", "tp_linear_bwd", "tpmlp_strerror",
+    "tpmlp_linear_workspace_size", "tp_linear_fwd", "tp_linear_bwd",
+    "tp_mlp_recompute_activation", "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
@@ -72,6 +73,8 @@ def lib() -> ctypes.CDLL:
             L.tp_linear_bwd.argtypes = [vp] * 6 + [i64, i64, i64, ctypes.c_int, ctypes.c_int,
                                                    ctypes.c_int, vp, sz, vp]
             L.tp_linear_bwd.restype = ctypes.c_int
+            L.tp_mlp_recompute_activation.argtypes = [vp, vp, i64, ctypes.c_int, ctypes.c_int, vp]
+            L.tp_mlp_recompute_activation.restype = ctypes.c_int
             L.tpmlp_strerror.argtypes = [ctypes.c_int]
             L.tpmlp_strerror.restype = ctypes.c_char_p
             L.tpmlp_last_device_status.argtypes = [vp]
@@ -363,3 +366,15 @@ def linear_backward(dY, X, W, p: int, split: str, *, out=None, workspace=None, s
                              ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
     _check(st, "tp_linear_bwd")
     return dX, dW, db
+
+
+def recompute_activation(H, *, out=None, activation: str = "gelu", stream=None):
+    """Y = act(H) elementwise (activation recompute before the backward)."""
+    if not H.is_cuda or not H.is_contiguous():
+        raise ValueError("H must be a contiguous CUDA tensor")
+    Y = torch.empty_like(H) if out is None else out
+    _need(Y, "Y", tuple(H.shape), H.dtype, H.device)
+    _check(lib().tp_mlp_recompute_activation(_ptr(H), _ptr(Y), H.numel(), _dtype_code(H),
+                                             _act_code(activation), _stream_ptr(H.device, stream)),
+           "tp_mlp_recompute_activation")
+    return Y

@@ -192,6 +192,56 @@ __global__ void eval_activation_kernel(const float* __restrict__ x, float* __res
     }
 }
 
+// Activation recompute: Y[i] = act(H[i]) for i < n. bf16 uses the
+// tensor-core epilogues' forms, fp32 the plain path's (CUDA erff / tanhf).
+// VEC: n % 8 == 0 and both pointers 16-byte aligned; 8 elements per
+// thread-iteration with 16-byte (bf16) or 2 × 16-byte (fp32) accesses.
+template <typename T, bool TANH, bool VEC>
+__global__ void __launch_bounds__(256) recompute_act_kernel(const T* __restrict__ H,
+                                                           T* __restrict__ Y, int64_t n) {
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    const int64_t first = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+    if constexpr (VEC) {
+        for (int64_t g = first; g < n / 8; g += stride) {
+            float f[8];
+            if constexpr (sizeof(T) == 2) {
+                unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(H) + g), f);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) f[i] = TANH ? gelu_tanh_fast(f[i]) : gelu_fast(f[i]);
+                uint4 o;
+                o.x = pack_bf16x2(f[0], f[1]);
+                o.y = pack_bf16x2(f[2], f[3]);
+                o.z = pack_bf16x2(f[4], f[5]);
+                o.w = pack_bf16x2(f[6], f[7]);
+                reinterpret_cast<uint4*>(Y)[g] = o;
+            } else {
+                const float4 lo = __ldg(reinterpret_cast<const float4*>(H) + 2 * g);
+                const float4 hi = __ldg(reinterpret_cast<const float4*>(H) + 2 * g + 1);
+                float4 a, b;
+                a.x = TANH ? gelu_tanh_f32(lo.x) : gelu_f32(lo.x);
+                a.y = TANH ? gelu_tanh_f32(lo.y) : gelu_f32(lo.y);
+                a.z = TANH ? gelu_tanh_f32(lo.z) : gelu_f32(lo.z);
+                a.w = TANH ? gelu_tanh_f32(lo.w) : gelu_f32(lo.w);
+                b.x = TANH ? gelu_tanh_f32(hi.x) : gelu_f32(hi.x);
+                b.y = TANH ? gelu_tanh_f32(hi.y) : gelu_f32(hi.y);
+                b.z = TANH ? gelu_tanh_f32(hi.z) : gelu_f32(hi.z);
+                b.w = TANH ? gelu_tanh_f32(hi.w) : gelu_f32(hi.w);
+                reinterpret_cast<float4*>(Y)[2 * g] = a;
+                reinterpret_cast<float4*>(Y)[2 * g + 1] = b;
+            }
+        }
+    } else {
+        for (int64_t i = first; i < n; i += stride) {
+            const float x = to_f32<T>(H[i]);
+            float y;
+            if constexpr (sizeof(T) == 2) y = TANH ? gelu_tanh_fast(x) : gelu_fast(x);
+            else y = TANH ? gelu_tanh_f32(x) : gelu_f32(x);
+            if constexpr (sizeof(T) == 2) Y[i] = __float2bfloat16_rn(y);
+            else Y[i] = y;
+        }
+    }
+}
+
 __global__ void zero_f32_kernel(float* __restrict__ p, int64_t n) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)

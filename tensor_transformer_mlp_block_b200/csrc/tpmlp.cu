@@ -141,14 +141,14 @@ tpmlp_status check_launch() {
 
 enum Kind : int {
     K_F1 = 0, K_F2, K_F2_RED, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_B5_RED, K_MISC,
-    K_L_FWD, K_L_FWD_RED, K_L_DB, K_L_DW, K_L_DX, K_L_DX_RED, K_COUNT
+    K_L_FWD, K_L_FWD_RED, K_L_DB, K_L_DW, K_L_DX, K_L_DX_RED, K_RECOMP, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "F2.split_reduce", "B1.db_colsum",
     "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
     "B5.dgrad_dX_shard_sum", "B5.split_reduce",       "misc",
     "L.fwd_gemm_bias",       "L.fwd_split_reduce",    "L.dbias_colsum",  "L.wgrad_dW",
-    "L.dgrad_dX",            "L.dgrad_split_reduce",
+    "L.dgrad_dX",            "L.dgrad_split_reduce",  "R.recompute_activation",
 };
 
 struct KindTotals {
@@ -887,6 +887,49 @@ tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* d
     cudaGetLastError();
     return linear_bwd_impl(dY, X, W, dX, dW, dbias, T, K, N, p, static_cast<int>(split), dt,
                            workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
+}
+
+tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpmlp_dtype dt,
+                                         tpmlp_activation act, void* stream) {
+    cudaGetLastError();
+    if (n < 0 || (dt != TPMLP_BF16 && dt != TPMLP_FP32)) return TPMLP_ERR_INVALID;
+    if (act != TPMLP_GELU_ERF && act != TPMLP_GELU_TANH) return TPMLP_ERR_INVALID;
+    if (n == 0) return TPMLP_OK;
+    if (!H || !Y) return TPMLP_ERR_INVALID;
+    const DeviceInfo* d = device_info();
+    if (d == nullptr) return TPMLP_ERR_CUDA;
+    if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t esize = dt == TPMLP_BF16 ? 2 : 4;
+    const bool vec = (n % 8 == 0) && aligned16(H) && aligned16(Y);
+    const int64_t work = vec ? n / 8 : n;
+    int64_t blocks = (work + 255) / 256;
+    const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    const bool tanh_form = (act == TPMLP_GELU_TANH);
+    return timed(K_RECOMP, 0.0, 2.0 * esize * static_cast<double>(n), st, [&] {
+        const unsigned nb = static_cast<unsigned>(blocks);
+        if (dt == TPMLP_BF16) {
+            const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(H);
+            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y);
+            if (vec)
+                tanh_form ? recompute_act_kernel<__nv_bfloat16, true, true><<<nb, 256, 0, st>>>(h, y, n)
+                          : recompute_act_kernel<__nv_bfloat16, false, true><<<nb, 256, 0, st>>>(h, y, n);
+            else
+                tanh_form ? recompute_act_kernel<__nv_bfloat16, true, false><<<nb, 256, 0, st>>>(h, y, n)
+                          : recompute_act_kernel<__nv_bfloat16, false, false><<<nb, 256, 0, st>>>(h, y, n);
+        } else {
+            const float* h = static_cast<const float*>(H);
+            float* y = static_cast<float*>(Y);
+            if (vec)
+                tanh_form ? recompute_act_kernel<float, true, true><<<nb, 256, 0, st>>>(h, y, n)
+                          : recompute_act_kernel<float, false, true><<<nb, 256, 0, st>>>(h, y, n);
+            else
+                tanh_form ? recompute_act_kernel<float, true, false><<<nb, 256, 0, st>>>(h, y, n)
+                          : recompute_act_kernel<float, false, false><<<nb, 256, 0, st>>>(h, y, n);
+        }
+        return check_launch();
+    });
 }
 
 const char* tpmlp_strerror(tpmlp_status s) {
