@@ -184,7 +184,19 @@ __global__ void eval_activation_kernel(const float* __restrict__ x, float* __res
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float v = x[i];
         switch (form) {
-            case 0: y[i] = gelu_fast(v); dy[i] = gelu_grad_fast(v); break;
+            case 0: {
+                // the packed pair (x[2k], x[2k+1]) as the epilogues form it,
+                // so both halves of the packed arithmetic are checked
+                const int64_t j = i ^ 1;
+                const float w = j < n ? x[j] : v;
+                const bool hi = (i & 1) != 0;
+                float p0, p1;
+                gelu_fast_x2(hi ? w : v, hi ? v : w, p0, p1);
+                y[i] = hi ? p1 : p0;
+                gelu_grad_fast_x2(hi ? w : v, hi ? v : w, p0, p1);
+                dy[i] = hi ? p1 : p0;
+                break;
+            }
             case 1: y[i] = gelu_f32(v); dy[i] = gelu_grad_f32(v); break;
             case 2: y[i] = gelu_tanh_fast(v); dy[i] = gelu_tanh_grad_fast(v); break;
             default: y[i] = gelu_tanh_f32(v); dy[i] = gelu_tanh_grad_f32(v); break;
@@ -207,7 +219,14 @@ __global__ void __launch_bounds__(256) recompute_act_kernel(const T* __restrict_
             if constexpr (sizeof(T) == 2) {
                 unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(H) + g), f);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) f[i] = TANH ? gelu_tanh_fast(f[i]) : gelu_fast(f[i]);
+                for (int i = 0; i < 8; i += 2) {
+                    if constexpr (TANH) {
+                        f[i] = gelu_tanh_fast(f[i]);
+                        f[i + 1] = gelu_tanh_fast(f[i + 1]);
+                    } else {
+                        gelu_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
+                    }
+                }
                 uint4 o;
                 o.x = pack_bf16x2(f[0], f[1]);
                 o.y = pack_bf16x2(f[2], f[3]);
@@ -234,8 +253,13 @@ __global__ void __launch_bounds__(256) recompute_act_kernel(const T* __restrict_
         for (int64_t i = first; i < n; i += stride) {
             const float x = to_f32<T>(H[i]);
             float y;
-            if constexpr (sizeof(T) == 2) y = TANH ? gelu_tanh_fast(x) : gelu_fast(x);
-            else y = TANH ? gelu_tanh_f32(x) : gelu_f32(x);
+            if constexpr (sizeof(T) == 2) {
+                float unused;
+                if constexpr (TANH) y = gelu_tanh_fast(x);
+                else gelu_fast_x2(x, x, y, unused);
+            } else {
+                y = TANH ? gelu_tanh_f32(x) : gelu_f32(x);
+            }
             if constexpr (sizeof(T) == 2) Y[i] = __float2bfloat16_rn(y);
             else Y[i] = y;
         }

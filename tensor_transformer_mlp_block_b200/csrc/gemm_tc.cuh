@@ -111,7 +111,41 @@ __device__ __forceinline__ float gelu_grad_f32(float x) {
     return cdf + x * pdf;
 }
 
-// Φ(x) and g = exp(−x²/2) for the tensor-core epilogues, from the rational
+// Two fp32 values in one 64-bit register: sm_100's fma.rn.f32x2 and
+// mul.rn.f32x2 work on both halves in one instruction, which halves the FP32
+// issue slots the epilogue's activation math takes.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_splat(float a) { return f2_pack(a, a); }
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& a, float& b) {
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t r;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+    uint64_t r;
+    asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+    return r;
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float exp2_approx(float x) {
+    float r;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+    return r;
+}
+
+// Φ(x) and g = exp(−x²/2) of two values at once for the
+// tensor-core epilogues, from the rational
 // approximation of erf by C. Hastings as printed in Abramowitz & Stegun,
 // Handbook of Mathematical Functions, eq. 7.1.26:
 //   erf(z) = 1 − (a1·t + a2·t² + a3·t³ + a4·t⁴ + a5·t⁵)·exp(−z²),
@@ -119,29 +153,40 @@ __device__ __forceinline__ float gelu_grad_f32(float x) {
 // With z = |x|/√2, exp(−z²) = exp(−x²/2) is the same factor the normal
 // density needs, so Φ and φ = g/√(2π) cost one exponential and one
 // reciprocal. Φ(−|x|) = ½·(1 − erf(z)); Φ(x) = 1 − Φ(−x).
-__device__ __forceinline__ void normal_cdf_and_gauss(float x, float& cdf, float& g) {
-    const float z = fabsf(x) * 0.70710678118654752f;
-    const float t = __fdividef(1.0f, fmaf(0.3275911f, z, 1.0f));
-    float poly = fmaf(1.061405429f, t, -1.453152027f);
-    poly = fmaf(poly, t, 1.421413741f);
-    poly = fmaf(poly, t, -0.284496736f);
-    poly = fmaf(poly, t, 0.254829592f);
-    poly *= t;
-    g = __expf(-0.5f * x * x);
-    const float tail = 0.5f * poly * g;  // Φ(−|x|)
-    cdf = x >= 0.0f ? 1.0f - tail : tail;
+// In the code the coefficients a1..a5 are halved, so that poly(t)·g is
+// Φ(−|x|) itself, and exp(−x²/2) = 2^(−x²·log2(e)/2).
+__device__ __forceinline__ void normal_cdf_and_gauss_x2(uint64_t x, float x0, float x1,
+                                                        uint64_t& cdf, uint64_t& g) {
+    const uint64_t z = f2_mul(f2_pack(fabsf(x0), fabsf(x1)), f2_splat(0.70710678118654752f));
+    float d0, d1;
+    f2_unpack(f2_fma(z, f2_splat(0.3275911f), f2_splat(1.0f)), d0, d1);
+    const uint64_t t = f2_pack(rcp_approx(d0), rcp_approx(d1));
+    uint64_t poly = f2_fma(f2_splat(0.5307027145f), t, f2_splat(-0.7265760135f));
+    poly = f2_fma(poly, t, f2_splat(0.7107068705f));
+    poly = f2_fma(poly, t, f2_splat(-0.142248368f));
+    poly = f2_fma(poly, t, f2_splat(0.127414796f));
+    poly = f2_mul(poly, t);
+    float m0, m1;
+    f2_unpack(f2_mul(f2_mul(x, x), f2_splat(-0.72134752044448170f)), m0, m1);
+    g = f2_pack(exp2_approx(m0), exp2_approx(m1));
+    float q0, q1;  // Φ(−|x|)
+    f2_unpack(f2_mul(poly, g), q0, q1);
+    cdf = f2_pack(x0 >= 0.0f ? 1.0f - q0 : q0, x1 >= 0.0f ? 1.0f - q1 : q1);
 }
 
-__device__ __forceinline__ float gelu_fast(float x) {
-    float cdf, g;
-    normal_cdf_and_gauss(x, cdf, g);
-    return x * cdf;
+// GeLU(x0), GeLU(x1) and GeLU′(x0), GeLU′(x1) of the tensor-core epilogues.
+__device__ __forceinline__ void gelu_fast_x2(float x0, float x1, float& y0, float& y1) {
+    const uint64_t x = f2_pack(x0, x1);
+    uint64_t cdf, g;
+    normal_cdf_and_gauss_x2(x, x0, x1, cdf, g);
+    f2_unpack(f2_mul(x, cdf), y0, y1);
 }
 
-__device__ __forceinline__ float gelu_grad_fast(float x) {
-    float cdf, g;
-    normal_cdf_and_gauss(x, cdf, g);
-    return fmaf(x * 0.39894228040143268f, g, cdf);
+__device__ __forceinline__ void gelu_grad_fast_x2(float x0, float x1, float& d0, float& d1) {
+    const uint64_t x = f2_pack(x0, x1);
+    uint64_t cdf, g;
+    normal_cdf_and_gauss_x2(x, x0, x1, cdf, g);
+    f2_unpack(f2_fma(f2_mul(x, f2_splat(0.39894228040143268f)), g, cdf), d0, d1);
 }
 
 // The tanh approximation of GeLU, ½·x·(1 + tanh u), u = √(2/π)·(x + 0.044715·x³),
@@ -179,15 +224,23 @@ __device__ __forceinline__ float gelu_tanh_grad_f32(float x) {
 
 // Activation of the tensor-core epilogues for epilogue kind EPI.
 template <int EPI>
-__device__ __forceinline__ float act_fast(float x) {
-    if constexpr (EpiTraits<EPI>::kTanh) return gelu_tanh_fast(x);
-    else return gelu_fast(x);
+__device__ __forceinline__ void act_fast_x2(float x0, float x1, float& y0, float& y1) {
+    if constexpr (EpiTraits<EPI>::kTanh) {
+        y0 = gelu_tanh_fast(x0);
+        y1 = gelu_tanh_fast(x1);
+    } else {
+        gelu_fast_x2(x0, x1, y0, y1);
+    }
 }
 
 template <int EPI>
-__device__ __forceinline__ float act_grad_fast(float x) {
-    if constexpr (EpiTraits<EPI>::kTanh) return gelu_tanh_grad_fast(x);
-    else return gelu_grad_fast(x);
+__device__ __forceinline__ void act_grad_fast_x2(float x0, float x1, float& d0, float& d1) {
+    if constexpr (EpiTraits<EPI>::kTanh) {
+        d0 = gelu_tanh_grad_fast(x0);
+        d1 = gelu_tanh_grad_fast(x1);
+    } else {
+        gelu_grad_fast_x2(x0, x1, d0, d1);
+    }
 }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
@@ -257,17 +310,24 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
                 if (row < g.M && c < g.N)
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
 #pragma unroll
-                for (int i = 0; i < 8; ++i) v[i] *= act_grad_fast<EPI>(hh[i]);
+                for (int i = 0; i < 8; i += 2) {
+                    float d0, d1;
+                    act_grad_fast_x2<EPI>(hh[i], hh[i + 1], d0, d1);
+                    f2_unpack(f2_mul(f2_pack(v[i], v[i + 1]), f2_pack(d0, d1)), v[i], v[i + 1]);
+                }
             }
             o0[q].x = pack_bf16x2(v[0], v[1]);
             o0[q].y = pack_bf16x2(v[2], v[3]);
             o0[q].z = pack_bf16x2(v[4], v[5]);
             o0[q].w = pack_bf16x2(v[6], v[7]);
             if constexpr (EpiTraits<EPI>::kAct) {
-                o1[q].x = pack_bf16x2(act_fast<EPI>(v[0]), act_fast<EPI>(v[1]));
-                o1[q].y = pack_bf16x2(act_fast<EPI>(v[2]), act_fast<EPI>(v[3]));
-                o1[q].z = pack_bf16x2(act_fast<EPI>(v[4]), act_fast<EPI>(v[5]));
-                o1[q].w = pack_bf16x2(act_fast<EPI>(v[6]), act_fast<EPI>(v[7]));
+                float y[8];
+#pragma unroll
+                for (int i = 0; i < 8; i += 2) act_fast_x2<EPI>(v[i], v[i + 1], y[i], y[i + 1]);
+                o1[q].x = pack_bf16x2(y[0], y[1]);
+                o1[q].y = pack_bf16x2(y[2], y[3]);
+                o1[q].z = pack_bf16x2(y[4], y[5]);
+                o1[q].w = pack_bf16x2(y[6], y[7]);
             }
         }
         if (lane == 0) bulk_wait_read0();
