@@ -51,8 +51,9 @@ def parse_args(argv=None):
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--activation", choices=["gelu", "gelu_tanh"], default="gelu",
                     help="MLP activation: exact GeLU (default) or its tanh approximation")
-    ap.add_argument("--recompute", action="store_true",
-                    help="activation recompute: rebuild Y from H before each backward")
+    ap.add_argument("--recompute", choices=["none", "activation", "hidden"], default="none",
+                    help="activation recompute before each backward: rebuild Y from H "
+                         "(activation) or H and Y from X (hidden)")
     ap.add_argument("--block", choices=["mlp", "attn-proj"], default="mlp",
                     help="mlp: the MLP block (default); attn-proj: the attention layer's "
                          "tensor-parallel projections (QKV split by columns, output by rows)")
@@ -289,8 +290,10 @@ def bench_ours(args, cfg, world, rank, local):
         dz = d["dZ"] if dz is None else dz
         binding.forward(x, d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, Z), workspace=ws,
                         activation=act)
-        if args.recompute:
+        if args.recompute == "activation":
             binding.recompute_activation(H, out=Y, activation=act)
+        elif args.recompute == "hidden":
+            binding.recompute_hidden(x, d["A"], d["a"], p, out=(H, Y), activation=act)
         binding.backward(dz, x, d["A"], d["B"], H, Y, p, out=gout, workspace=ws, activation=act)
 
     working_set = sum(t.numel() * t.element_size() for t in [*d.values(), H, Y, Z, *gout.values()])
@@ -463,6 +466,10 @@ def e2e_measure(args, cfg, inp, d, H, Y, Z, gout, ws, p, T, h, dt, dev, stream, 
             binding.forward(xin[b], d["A"], d["a"], d["B"], d["b"], p, out=(H, Y, zout[b]),
                             workspace=ws, activation=act)
             gout["dX"] = dxout[b]
+            if args.recompute == "activation":
+                binding.recompute_activation(H, out=Y, activation=act)
+            elif args.recompute == "hidden":
+                binding.recompute_hidden(xin[b], d["A"], d["a"], p, out=(H, Y), activation=act)
             binding.backward(dzin[b], xin[b], d["A"], d["B"], H, Y, p, out=gout, workspace=ws,
                              activation=act)
             ev_comp[b].record(stream)
@@ -500,8 +507,10 @@ def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, la
     else:
         if args.activation != "gelu":
             workload += f" ({args.activation})"
-        if args.recompute:
-            workload += " with activation recompute"
+        if args.recompute == "activation":
+            workload += " with activation recompute (Y from H)"
+        elif args.recompute == "hidden":
+            workload += " with activation recompute (H and Y from X)"
     metric = METRIC if args.block == "mlp" else \
         "TP attention projections fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
     return {

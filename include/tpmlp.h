@@ -153,6 +153,16 @@ tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* d
 tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpmlp_dtype dt,
                                          tpmlp_activation act, void* stream);
 
+/* Activation recompute from the block's input (same section): a caller that
+ * keeps only X rebuilds H = X·A + a and Y = act(H) before the backward, the
+ * forward's first product (column split, no shard sum) without the second.
+ * Arguments, layouts, requirements and errors as tp_mlp_fwd_ex, without B,
+ * b, Z and the workspace (this product needs none). H and Y are bitwise
+ * those of tp_mlp_fwd_ex on the same inputs. Costs 2·T·h·F flops. */
+tpmlp_status tp_mlp_recompute_hidden(const void* X, const void* A, const void* a, void* H, void* Y,
+                                     int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
+                                     tpmlp_activation act, void* stream);
+
 /* Static, NUL-terminated description of a status code. */
 const char* tpmlp_strerror(tpmlp_status s);
 

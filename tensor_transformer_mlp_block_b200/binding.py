@@ -23,7 +23,7 @@ ACTIVATIONS = {"gelu": 0, "gelu_tanh": 1}
 EXPORTS = (
     "tpmlp_workspace_size", "tp_mlp_fwd", "tp_mlp_bwd", "tp_mlp_fwd_ex", "tp_mlp_bwd_ex",
     "tpmlp_linear_workspace_size", "tp_linear_fwd", "tp_linear_bwd",
-    "tp_mlp_recompute_activation", "tpmlp_strerror",
+    "tp_mlp_recompute_activation", "tp_mlp_recompute_hidden", "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
@@ -75,6 +75,9 @@ def lib() -> ctypes.CDLL:
             L.tp_linear_bwd.restype = ctypes.c_int
             L.tp_mlp_recompute_activation.argtypes = [vp, vp, i64, ctypes.c_int, ctypes.c_int, vp]
             L.tp_mlp_recompute_activation.restype = ctypes.c_int
+            L.tp_mlp_recompute_hidden.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ctypes.c_int,
+                                                  ctypes.c_int, ctypes.c_int, vp]
+            L.tp_mlp_recompute_hidden.restype = ctypes.c_int
             L.tpmlp_strerror.argtypes = [ctypes.c_int]
             L.tpmlp_strerror.restype = ctypes.c_char_p
             L.tpmlp_last_device_status.argtypes = [vp]
@@ -366,6 +369,30 @@ def linear_backward(dY, X, W, p: int, split: str, *, out=None, workspace=None, s
                              ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
     _check(st, "tp_linear_bwd")
     return dX, dW, db
+
+
+def recompute_hidden(X, A, a, p: int, *, out=None, activation: str = "gelu", stream=None):
+    """H = X·A + a and Y = act(H) (the forward's first product alone), for
+    a caller that keeps only X. Returns (H, Y); `out` may supply them."""
+    T, h = X.shape
+    F = A.shape[1]
+    dt, dev = X.dtype, X.device
+    _need(X, "X", (T, h), dt, dev)
+    _need(A, "A", (h, F), dt, dev)
+    if a is not None:
+        _need(a, "a", (F,), dt, dev)
+    if out is None:
+        H = torch.empty((T, F), dtype=dt, device=dev)
+        Y = torch.empty((T, F), dtype=dt, device=dev)
+    else:
+        H, Y = out
+        _need(H, "H", (T, F), dt, dev)
+        _need(Y, "Y", (T, F), dt, dev)
+    _check(lib().tp_mlp_recompute_hidden(_ptr(X), _ptr(A), _ptr(a), _ptr(H), _ptr(Y), T, h, F,
+                                         int(p), _dtype_code(X), _act_code(activation),
+                                         _stream_ptr(dev, stream)),
+           "tp_mlp_recompute_hidden")
+    return H, Y
 
 
 def recompute_activation(H, *, out=None, activation: str = "gelu", stream=None):

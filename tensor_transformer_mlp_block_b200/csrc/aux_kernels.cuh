@@ -206,47 +206,73 @@ __global__ void eval_activation_kernel(const float* __restrict__ x, float* __res
 
 // Activation recompute: Y[i] = act(H[i]) for i < n. bf16 uses the
 // tensor-core epilogues' forms, fp32 the plain path's (CUDA erff / tanhf).
-// VEC: n % 8 == 0 and both pointers 16-byte aligned; 8 elements per
-// thread-iteration with 16-byte (bf16) or 2 × 16-byte (fp32) accesses.
+template <bool TANH>
+__device__ __forceinline__ uint4 act_bf16x8(uint4 raw) {
+    float f[8];
+    unpack_bf16x8(raw, f);
+#pragma unroll
+    for (int i = 0; i < 8; i += 2) {
+        if constexpr (TANH) {
+            f[i] = gelu_tanh_fast(f[i]);
+            f[i + 1] = gelu_tanh_fast(f[i + 1]);
+        } else {
+            gelu_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
+        }
+    }
+    uint4 o;
+    o.x = pack_bf16x2(f[0], f[1]);
+    o.y = pack_bf16x2(f[2], f[3]);
+    o.z = pack_bf16x2(f[4], f[5]);
+    o.w = pack_bf16x2(f[6], f[7]);
+    return o;
+}
+
+template <bool TANH>
+__device__ __forceinline__ float4 act_f32x4(float4 v) {
+    v.x = TANH ? gelu_tanh_f32(v.x) : gelu_f32(v.x);
+    v.y = TANH ? gelu_tanh_f32(v.y) : gelu_f32(v.y);
+    v.z = TANH ? gelu_tanh_f32(v.z) : gelu_f32(v.z);
+    v.w = TANH ? gelu_tanh_f32(v.w) : gelu_f32(v.w);
+    return v;
+}
+
+// VEC: n % 8 == 0 and both pointers 16-byte aligned. 8 elements form one
+// group (16 bytes of bf16, 32 of fp32); a thread-iteration takes two groups a
+// grid stride apart and issues both loads before computing either, so that
+// more bytes are in flight per SM.
 template <typename T, bool TANH, bool VEC>
-__global__ void __launch_bounds__(256) recompute_act_kernel(const T* __restrict__ H,
+__global__ void __launch_bounds__(256, 8) recompute_act_kernel(const T* __restrict__ H,
                                                            T* __restrict__ Y, int64_t n) {
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t first = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if constexpr (VEC) {
-        for (int64_t g = first; g < n / 8; g += stride) {
-            float f[8];
+        const int64_t groups = n / 8;
+        for (int64_t g = first; g < groups; g += 2 * stride) {
+            const int64_t g2 = g + stride;
+            const bool second = g2 < groups;
             if constexpr (sizeof(T) == 2) {
-                unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(H) + g), f);
-#pragma unroll
-                for (int i = 0; i < 8; i += 2) {
-                    if constexpr (TANH) {
-                        f[i] = gelu_tanh_fast(f[i]);
-                        f[i + 1] = gelu_tanh_fast(f[i + 1]);
-                    } else {
-                        gelu_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
-                    }
-                }
-                uint4 o;
-                o.x = pack_bf16x2(f[0], f[1]);
-                o.y = pack_bf16x2(f[2], f[3]);
-                o.z = pack_bf16x2(f[4], f[5]);
-                o.w = pack_bf16x2(f[6], f[7]);
-                reinterpret_cast<uint4*>(Y)[g] = o;
+                const uint4* h = reinterpret_cast<const uint4*>(H);
+                uint4* y = reinterpret_cast<uint4*>(Y);
+                const uint4 r0 = __ldg(h + g);
+                uint4 r1 = make_uint4(0, 0, 0, 0);
+                if (second) r1 = __ldg(h + g2);
+                y[g] = act_bf16x8<TANH>(r0);
+                if (second) y[g2] = act_bf16x8<TANH>(r1);
             } else {
-                const float4 lo = __ldg(reinterpret_cast<const float4*>(H) + 2 * g);
-                const float4 hi = __ldg(reinterpret_cast<const float4*>(H) + 2 * g + 1);
-                float4 a, b;
-                a.x = TANH ? gelu_tanh_f32(lo.x) : gelu_f32(lo.x);
-                a.y = TANH ? gelu_tanh_f32(lo.y) : gelu_f32(lo.y);
-                a.z = TANH ? gelu_tanh_f32(lo.z) : gelu_f32(lo.z);
-                a.w = TANH ? gelu_tanh_f32(lo.w) : gelu_f32(lo.w);
-                b.x = TANH ? gelu_tanh_f32(hi.x) : gelu_f32(hi.x);
-                b.y = TANH ? gelu_tanh_f32(hi.y) : gelu_f32(hi.y);
-                b.z = TANH ? gelu_tanh_f32(hi.z) : gelu_f32(hi.z);
-                b.w = TANH ? gelu_tanh_f32(hi.w) : gelu_f32(hi.w);
-                reinterpret_cast<float4*>(Y)[2 * g] = a;
-                reinterpret_cast<float4*>(Y)[2 * g + 1] = b;
+                const float4* h = reinterpret_cast<const float4*>(H);
+                float4* y = reinterpret_cast<float4*>(Y);
+                const float4 a0 = __ldg(h + 2 * g), a1 = __ldg(h + 2 * g + 1);
+                float4 b0 = make_float4(0, 0, 0, 0), b1 = b0;
+                if (second) {
+                    b0 = __ldg(h + 2 * g2);
+                    b1 = __ldg(h + 2 * g2 + 1);
+                }
+                y[2 * g] = act_f32x4<TANH>(a0);
+                y[2 * g + 1] = act_f32x4<TANH>(a1);
+                if (second) {
+                    y[2 * g2] = act_f32x4<TANH>(b0);
+                    y[2 * g2 + 1] = act_f32x4<TANH>(b1);
+                }
             }
         }
     } else {

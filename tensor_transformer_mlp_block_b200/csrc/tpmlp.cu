@@ -419,6 +419,30 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Blocks of `threads` threads that the device holds at once for KERNEL (per
+// SM from the occupancy calculator, cached per kernel). Grid-stride kernels
+// launch no more than this, so that no block waits for a second wave.
+template <auto KERNEL>
+int64_t resident_blocks(int threads) {
+    static std::atomic<int> cached{0};
+    int per_sm = cached.load(std::memory_order_relaxed);
+    if (per_sm == 0) {
+        if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, KERNEL, threads, 0) !=
+                cudaSuccess || per_sm < 1) {
+            cudaGetLastError();
+            per_sm = 1;
+        }
+        cached.store(per_sm, std::memory_order_relaxed);
+    }
+    const DeviceInfo* d = device_info();
+    return static_cast<int64_t>(per_sm) * (d ? d->num_sms : 148);
+}
+
+int64_t clamp_grid(int64_t blocks, int64_t cap) {
+    if (blocks > cap) blocks = cap;
+    return blocks < 1 ? 1 : blocks;
+}
+
 template <typename T>
 tpmlp_status colsum_launch(const T* X, int64_t R, int64_t C, int64_t chunks, float* partial,
                            float* out, cudaStream_t st) {
@@ -445,12 +469,9 @@ tpmlp_status colsum(int kind, const T* X, int64_t R, int64_t C, int64_t chunks, 
 
 tpmlp_status reduce_splits_launch(const float* ws, int splits, int64_t M, int64_t N,
                                   const void* bias, void* out, cudaStream_t st) {
-    const DeviceInfo* dev = device_info();
     const int64_t groups = M * (N / 8);
-    int64_t blocks = (groups + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(dev ? dev->num_sms : 148) * 8;
-    if (blocks > cap) blocks = cap;
-    if (blocks < 1) blocks = 1;
+    const int64_t blocks =
+        clamp_grid((groups + 255) / 256, resident_blocks<reduce_splits_bf16_kernel>(256));
     reduce_splits_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
         ws, splits, M * N, static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(out),
         M, N);
@@ -463,11 +484,22 @@ tpmlp_status reduce_splits(int kind, const float* ws, int splits, int64_t M, int
                  [&] { return reduce_splits_launch(ws, splits, M, N, bias, out, st); });
 }
 
+// One launch of recompute_act_kernel over n elements: a thread-iteration
+// takes two 8-element groups (VEC) or one element; no more blocks than the
+// device holds at once.
+template <typename T, bool TANH, bool VEC>
+void launch_recompute(const void* H, void* Y, int64_t n, cudaStream_t st) {
+    const int64_t work = VEC ? (n / 8 + 1) / 2 : n;
+    const unsigned nb = static_cast<unsigned>(
+        clamp_grid((work + 255) / 256, resident_blocks<recompute_act_kernel<T, TANH, VEC>>(256)));
+    recompute_act_kernel<T, TANH, VEC>
+        <<<nb, 256, 0, st>>>(static_cast<const T*>(H), static_cast<T*>(Y), n);
+}
+
 tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st) {
     if (n <= 0) return TPMLP_OK;
     return timed(K_MISC, 0.0, 4.0 * n, st, [&] {
-        int64_t blocks = (n + 255) / 256;
-        if (blocks > 1184) blocks = 1184;
+        const int64_t blocks = clamp_grid((n + 255) / 256, resident_blocks<zero_f32_kernel>(256));
         zero_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, n);
         return check_launch();
     });
@@ -480,7 +512,7 @@ tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st) {
     } while (0)
 
 tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl,
-                           void* ws, size_t ws_bytes) {
+                           void* ws, size_t ws_bytes, bool need_ws = true) {
     if (!make_plan(T, h, F, p, dt, pl)) return TPMLP_ERR_INVALID;
     // the kernels index rows, columns and tiles with 32-bit integers
     if (T >= (int64_t(1) << 31) || h >= (int64_t(1) << 31) || F >= (int64_t(1) << 31))
@@ -488,7 +520,8 @@ tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype d
     const DeviceInfo* d = device_info();
     if (d == nullptr) return TPMLP_ERR_CUDA;
     if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
-    if (pl->total > 0 && (ws == nullptr || ws_bytes < pl->total)) return TPMLP_ERR_WORKSPACE;
+    if (need_ws && pl->total > 0 && (ws == nullptr || ws_bytes < pl->total))
+        return TPMLP_ERR_WORKSPACE;
     if (ws != nullptr && !aligned16(ws)) return TPMLP_ERR_ALIGN;
     return TPMLP_OK;
 }
@@ -537,7 +570,8 @@ tpmlp_status lin_checks(int64_t T, int64_t K, int64_t N, int p, int split, tpmlp
     const DeviceInfo* d = device_info();
     if (d == nullptr) return TPMLP_ERR_CUDA;
     if (d->cc_major != 10) return TPMLP_ERR_UNSUPPORTED;
-    if (pl->total > 0 && (ws == nullptr || ws_bytes < pl->total)) return TPMLP_ERR_WORKSPACE;
+    if (pl->total > 0 && (ws == nullptr || ws_bytes < pl->total))
+        return TPMLP_ERR_WORKSPACE;
     if (ws != nullptr && !aligned16(ws)) return TPMLP_ERR_ALIGN;
     return TPMLP_OK;
 }
@@ -639,15 +673,18 @@ tpmlp_status linear_bwd_impl(const void* dY, const void* X, const void* W, void*
 }
 
 // Forward with activation epilogue EPI_ACT (EPI_GELU or EPI_GELU_TANH).
+// with_f2 = false runs F1 alone (H and Y from X; B, b and Z unused).
 template <int EPI_ACT>
 tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B, const void* b,
                       void* H, void* Y, void* Z, int64_t T, int64_t h, int64_t F, int p,
-                      tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream) {
+                      tpmlp_dtype dt, void* workspace, size_t workspace_bytes, void* stream,
+                      bool with_f2 = true) {
     cudaGetLastError();  // start from a clean (non-sticky) error state
     Plan pl;
-    TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes));
+    TPMLP_TRY(common_checks(T, h, F, p, dt, &pl, workspace, workspace_bytes, with_f2));
     if (T == 0) return TPMLP_OK;
-    if (!X || !A || !B || !H || !Y || !Z) return TPMLP_ERR_INVALID;
+    if (!X || !A || !H || !Y) return TPMLP_ERR_INVALID;
+    if (with_f2 && (!B || !Z)) return TPMLP_ERR_INVALID;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     if (pl.tc) {
         for (const void* q : {X, A, a, B, b, static_cast<const void*>(H), static_cast<const void*>(Y),
@@ -661,6 +698,7 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
         g1.ld_out = F;
         g1.bias = static_cast<const __nv_bfloat16*>(a);
         TPMLP_TRY((gemm_tc<256, false, true, EPI_ACT>(K_F1, X, A, iT, iF, ih, 1, g1, st)));
+        if (!with_f2) return TPMLP_OK;
         // F2: Z = Σ_i Y_i·B_i + b. Aop = Y [T][F] (K-major), Bop = B [F][h] (MN-major).
         GemmArgs g2{};
         if (pl.splits == 1) {
@@ -691,10 +729,10 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
     s2.out0 = Z; s2.ld_out = h; s2.bias = b;
     if (dt == TPMLP_FP32) {
         TPMLP_TRY((gemm_simt<float, EPI_ACT>(K_F1, s1, st)));
-        TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_F2, s2, st)));
+        if (with_f2) TPMLP_TRY((gemm_simt<float, EPI_BIAS>(K_F2, s2, st)));
     } else {
         TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_ACT>(K_F1, s1, st)));
-        TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_F2, s2, st)));
+        if (with_f2) TPMLP_TRY((gemm_simt<__nv_bfloat16, EPI_BIAS>(K_F2, s2, st)));
     }
     return TPMLP_OK;
 }
@@ -889,6 +927,20 @@ tpmlp_status tp_linear_bwd(const void* dY, const void* X, const void* W, void* d
                            workspace, workspace_bytes, static_cast<cudaStream_t>(stream));
 }
 
+tpmlp_status tp_mlp_recompute_hidden(const void* X, const void* A, const void* a, void* H, void* Y,
+                                     int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt,
+                                     tpmlp_activation act, void* stream) {
+    switch (act) {
+        case TPMLP_GELU_ERF:
+            return fwd_impl<EPI_GELU>(X, A, a, nullptr, nullptr, H, Y, nullptr, T, h, F, p, dt,
+                                      nullptr, 0, stream, false);
+        case TPMLP_GELU_TANH:
+            return fwd_impl<EPI_GELU_TANH>(X, A, a, nullptr, nullptr, H, Y, nullptr, T, h, F, p,
+                                           dt, nullptr, 0, stream, false);
+    }
+    return TPMLP_ERR_INVALID;
+}
+
 tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpmlp_dtype dt,
                                          tpmlp_activation act, void* stream) {
     cudaGetLastError();
@@ -902,31 +954,23 @@ tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpml
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t esize = dt == TPMLP_BF16 ? 2 : 4;
     const bool vec = (n % 8 == 0) && aligned16(H) && aligned16(Y);
-    const int64_t work = vec ? n / 8 : n;
-    int64_t blocks = (work + 255) / 256;
-    const int64_t cap = static_cast<int64_t>(d->num_sms) * 8;
-    if (blocks > cap) blocks = cap;
     const bool tanh_form = (act == TPMLP_GELU_TANH);
     return timed(K_RECOMP, 0.0, 2.0 * esize * static_cast<double>(n), st, [&] {
-        const unsigned nb = static_cast<unsigned>(blocks);
+        using B = __nv_bfloat16;
         if (dt == TPMLP_BF16) {
-            const __nv_bfloat16* h = static_cast<const __nv_bfloat16*>(H);
-            __nv_bfloat16* y = static_cast<__nv_bfloat16*>(Y);
             if (vec)
-                tanh_form ? recompute_act_kernel<__nv_bfloat16, true, true><<<nb, 256, 0, st>>>(h, y, n)
-                          : recompute_act_kernel<__nv_bfloat16, false, true><<<nb, 256, 0, st>>>(h, y, n);
+                tanh_form ? launch_recompute<B, true, true>(H, Y, n, st)
+                          : launch_recompute<B, false, true>(H, Y, n, st);
             else
-                tanh_form ? recompute_act_kernel<__nv_bfloat16, true, false><<<nb, 256, 0, st>>>(h, y, n)
-                          : recompute_act_kernel<__nv_bfloat16, false, false><<<nb, 256, 0, st>>>(h, y, n);
+                tanh_form ? launch_recompute<B, true, false>(H, Y, n, st)
+                          : launch_recompute<B, false, false>(H, Y, n, st);
         } else {
-            const float* h = static_cast<const float*>(H);
-            float* y = static_cast<float*>(Y);
             if (vec)
-                tanh_form ? recompute_act_kernel<float, true, true><<<nb, 256, 0, st>>>(h, y, n)
-                          : recompute_act_kernel<float, false, true><<<nb, 256, 0, st>>>(h, y, n);
+                tanh_form ? launch_recompute<float, true, true>(H, Y, n, st)
+                          : launch_recompute<float, false, true>(H, Y, n, st);
             else
-                tanh_form ? recompute_act_kernel<float, true, false><<<nb, 256, 0, st>>>(h, y, n)
-                          : recompute_act_kernel<float, false, false><<<nb, 256, 0, st>>>(h, y, n);
+                tanh_form ? launch_recompute<float, true, false>(H, Y, n, st)
+                          : launch_recompute<float, false, false>(H, Y, n, st);
         }
         return check_launch();
     });

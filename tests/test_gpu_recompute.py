@@ -64,3 +64,48 @@ def test_recompute_errors_and_empty():
         binding.recompute_activation(H, activation="relu")
     L = binding.lib()
     assert L.tp_mlp_recompute_activation(H.data_ptr(), H.data_ptr(), -1, 0, 0, None) == binding.ERR_INVALID
+
+
+@pytest.mark.parametrize("T,h,F,p,dtype,act", [
+    (300, 200, 520, 2, "bf16", "gelu"),        # tensor-core path, ragged tails
+    (256, 128, 512, 4, "bf16", "gelu_tanh"),
+    (37, 12, 44, 2, "bf16", "gelu"),           # plain path (h, F not multiples of 8)
+    (512, 12, 48, 2, "fp32", "gelu"),          # fp32 toy shape
+])
+def test_recompute_hidden_is_the_forward_first_product(T, h, F, p, dtype, act):
+    """H and Y rebuilt from X are bitwise those of the forward."""
+    from tensor_transformer_mlp_block_b200.inputs import make_shape
+    inp = make_shape(T, h, F, dtype, seed_offset=T + F)
+    d = {k: v.cuda() for k, v in inp.items()}
+    H, Y, _ = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p, activation=act)
+    H2, Y2 = binding.recompute_hidden(d["X"], d["A"], d["a"], p, activation=act)
+    torch.cuda.synchronize()
+    assert torch.equal(H, H2) and torch.equal(Y, Y2)
+
+
+def test_backward_on_hidden_recomputed_from_x():
+    """fwd -> drop H and Y -> rebuild both from X -> bwd: gradients match the oracle."""
+    cfg = configs.get("gpt2-small")
+    inp = make_inputs(cfg)
+    d = {k: v.cuda() for k, v in inp.items()}
+    _, _, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], cfg.p)
+    H, Y = binding.recompute_hidden(d["X"], d["A"], d["a"], cfg.p)
+    g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, cfg.p)
+    torch.cuda.synchronize()
+    got = dict(H=H.cpu(), Y=Y.cpu(), Z=Z.cpu(), **{k: v.cpu() for k, v in g.items()})
+    compare_full(got, oracle_full(inp), "bf16")
+
+
+def test_recompute_hidden_errors():
+    X = torch.zeros((64, 64), dtype=torch.bfloat16, device="cuda")
+    A = torch.zeros((64, 96), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(binding.TPMLPError) as e:
+        binding.recompute_hidden(X, A, None, 5)  # 96 % 5 != 0
+    assert e.value.status == binding.ERR_INVALID
+    with pytest.raises(ValueError):
+        binding.recompute_hidden(X, A, None, 2, activation="relu")
+    L = binding.lib()
+    assert L.tp_mlp_recompute_hidden(None, A.data_ptr(), None, X.data_ptr(), X.data_ptr(),
+                                     64, 64, 96, 2, 0, 0, None) == binding.ERR_INVALID
+    H, Y = binding.recompute_hidden(X[:0], A, None, 2)
+    assert H.shape == (0, 96) and Y.shape == (0, 96)
