@@ -211,7 +211,7 @@ uint64_t tpmlp_launch_count(void);
  *           |error| ≤ 1.5e−7) sharing exp(−x²/2) with φ(x);
  *   form 1: exact GeLU through CUDA's erff and expf (the plain path);
  *   form 2: the tanh approximation as the tensor-core epilogues compute it,
- *           tanh u = 1 − 2/(1 + exp(2u));
+ *           ½(1 + tanh u) = 1/(1 + exp(−2u));
  *   form 3: the tanh approximation through CUDA's tanhf (the plain path).
  * Returns TPMLP_ERR_INVALID for n < 0, null pointers or another form. */
 tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t n, int form,

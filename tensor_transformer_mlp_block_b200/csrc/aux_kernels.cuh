@@ -177,29 +177,36 @@ __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restri
 // GeLU and GeLU′ of n values with each form the library uses:
 // 0 = exact GeLU as in the tensor-core epilogues (Hastings erf), 1 = exact
 // GeLU through CUDA's erff/expf, 2 = tanh form as in the tensor-core
-// epilogues (exp-based tanh), 3 = tanh form through CUDA's tanhf.
+// epilogues (½(1 + tanh u) as a logistic function of 2u), 3 = tanh form
+// through CUDA's tanhf. Forms 0 and 2 run in packed pairs like the epilogues.
 __global__ void eval_activation_kernel(const float* __restrict__ x, float* __restrict__ y,
                                        float* __restrict__ dy, int64_t n, int form) {
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
         const float v = x[i];
-        switch (form) {
-            case 0: {
-                // the packed pair (x[2k], x[2k+1]) as the epilogues form it,
-                // so both halves of the packed arithmetic are checked
-                const int64_t j = i ^ 1;
-                const float w = j < n ? x[j] : v;
-                const bool hi = (i & 1) != 0;
-                float p0, p1;
-                gelu_fast_x2(hi ? w : v, hi ? v : w, p0, p1);
-                y[i] = hi ? p1 : p0;
-                gelu_grad_fast_x2(hi ? w : v, hi ? v : w, p0, p1);
-                dy[i] = hi ? p1 : p0;
-                break;
+        if (form == 0 || form == 2) {
+            // the packed pair (x[2k], x[2k+1]) as the epilogues form it, so
+            // both halves of the packed arithmetic are checked
+            const int64_t j = i ^ 1;
+            const float w = j < n ? x[j] : v;
+            const bool hi = (i & 1) != 0;
+            const float a = hi ? w : v, b = hi ? v : w;
+            float p0, p1, q0, q1;
+            if (form == 0) {
+                gelu_fast_x2(a, b, p0, p1);
+                gelu_grad_fast_x2(a, b, q0, q1);
+            } else {
+                gelu_tanh_fast_x2(a, b, p0, p1);
+                gelu_tanh_grad_fast_x2(a, b, q0, q1);
             }
-            case 1: y[i] = gelu_f32(v); dy[i] = gelu_grad_f32(v); break;
-            case 2: y[i] = gelu_tanh_fast(v); dy[i] = gelu_tanh_grad_fast(v); break;
-            default: y[i] = gelu_tanh_f32(v); dy[i] = gelu_tanh_grad_f32(v); break;
+            y[i] = hi ? p1 : p0;
+            dy[i] = hi ? q1 : q0;
+        } else if (form == 1) {
+            y[i] = gelu_f32(v);
+            dy[i] = gelu_grad_f32(v);
+        } else {
+            y[i] = gelu_tanh_f32(v);
+            dy[i] = gelu_tanh_grad_f32(v);
         }
     }
 }
@@ -212,12 +219,8 @@ __device__ __forceinline__ uint4 act_bf16x8(uint4 raw) {
     unpack_bf16x8(raw, f);
 #pragma unroll
     for (int i = 0; i < 8; i += 2) {
-        if constexpr (TANH) {
-            f[i] = gelu_tanh_fast(f[i]);
-            f[i + 1] = gelu_tanh_fast(f[i + 1]);
-        } else {
-            gelu_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
-        }
+        if constexpr (TANH) gelu_tanh_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
+        else gelu_fast_x2(f[i], f[i + 1], f[i], f[i + 1]);
     }
     uint4 o;
     o.x = pack_bf16x2(f[0], f[1]);
@@ -281,7 +284,7 @@ __global__ void __launch_bounds__(256, 8) recompute_act_kernel(const T* __restri
             float y;
             if constexpr (sizeof(T) == 2) {
                 float unused;
-                if constexpr (TANH) y = gelu_tanh_fast(x);
+                if constexpr (TANH) gelu_tanh_fast_x2(x, x, y, unused);
                 else gelu_fast_x2(x, x, y, unused);
             } else {
                 y = TANH ? gelu_tanh_f32(x) : gelu_f32(x);

@@ -190,23 +190,37 @@ __device__ __forceinline__ void gelu_grad_fast_x2(float x0, float x1, float& d0,
 }
 
 // The tanh approximation of GeLU, ½·x·(1 + tanh u), u = √(2/π)·(x + 0.044715·x³),
-// with tanh u = 1 − 2 / (1 + exp(2u)) (one exponential and one reciprocal;
-// exp(2u) = ∞ gives tanh u = 1 and exp(2u) = 0 gives −1, as they should).
-__device__ __forceinline__ float tanh_via_exp(float u) {
-    return 1.0f - __fdividef(2.0f, 1.0f + __expf(2.0f * u));
+// for two values at once. ½·(1 + tanh u) is the logistic function
+// s = 1/(1 + exp(−2u)), so GeLU_tanh(x) = x·s: one exp2 and one reciprocal,
+// with no cancellation for negative x (exp(−2u) = ∞ gives s = 0).
+// The derivative, ½(1 + tanh u) + ½·x·(1 − tanh² u)·u′, is
+// s + x·s·(1 − s)·2u′ with 2u′ = 2√(2/π)·(1 + 3·0.044715·x²).
+__device__ __forceinline__ uint64_t logistic_2u_x2(uint64_t x, uint64_t x2) {
+    // −2u·log2(e) = x·(1 + 0.044715·x²)·(−2√(2/π)·log2(e))
+    const uint64_t inner = f2_fma(x2, f2_splat(0.044715f), f2_splat(1.0f));
+    float m0, m1;
+    f2_unpack(f2_mul(f2_mul(x, inner), f2_splat(-2.3022082f)), m0, m1);
+    const uint64_t e = f2_pack(exp2_approx(m0), exp2_approx(m1));
+    float d0, d1;
+    f2_unpack(f2_fma(e, f2_splat(1.0f), f2_splat(1.0f)), d0, d1);
+    return f2_pack(rcp_approx(d0), rcp_approx(d1));
 }
 
-__device__ __forceinline__ float gelu_tanh_fast(float x) {
-    const float u = 0.79788456080286536f * x * fmaf(0.044715f * x, x, 1.0f);
-    return 0.5f * x * (1.0f + tanh_via_exp(u));
+__device__ __forceinline__ void gelu_tanh_fast_x2(float x0, float x1, float& y0, float& y1) {
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t s = logistic_2u_x2(x, f2_mul(x, x));
+    f2_unpack(f2_mul(x, s), y0, y1);
 }
 
-// ½(1 + tanh u) + ½·x·(1 − tanh² u)·√(2/π)·(1 + 3·0.044715·x²)
-__device__ __forceinline__ float gelu_tanh_grad_fast(float x) {
-    const float u = 0.79788456080286536f * x * fmaf(0.044715f * x, x, 1.0f);
-    const float th = tanh_via_exp(u);
-    const float du = 0.79788456080286536f * fmaf(0.134145f * x, x, 1.0f);
-    return fmaf(0.5f * x * du, fmaf(-th, th, 1.0f), 0.5f * (1.0f + th));
+__device__ __forceinline__ void gelu_tanh_grad_fast_x2(float x0, float x1, float& d0, float& d1) {
+    const uint64_t x = f2_pack(x0, x1);
+    const uint64_t x2 = f2_mul(x, x);
+    const uint64_t s = logistic_2u_x2(x, x2);
+    // 2u′ = 2√(2/π) + 2√(2/π)·0.134145·x²
+    const uint64_t du2 = f2_fma(x2, f2_splat(0.21406445f), f2_splat(1.5957691f));
+    const uint64_t one_minus_s = f2_fma(s, f2_splat(-1.0f), f2_splat(1.0f));
+    const uint64_t t = f2_mul(f2_mul(x, s), one_minus_s);
+    f2_unpack(f2_fma(t, du2, s), d0, d1);
 }
 
 // The same two functions through CUDA's tanhf (the plain path).
@@ -226,8 +240,7 @@ __device__ __forceinline__ float gelu_tanh_grad_f32(float x) {
 template <int EPI>
 __device__ __forceinline__ void act_fast_x2(float x0, float x1, float& y0, float& y1) {
     if constexpr (EpiTraits<EPI>::kTanh) {
-        y0 = gelu_tanh_fast(x0);
-        y1 = gelu_tanh_fast(x1);
+        gelu_tanh_fast_x2(x0, x1, y0, y1);
     } else {
         gelu_fast_x2(x0, x1, y0, y1);
     }
@@ -236,8 +249,7 @@ __device__ __forceinline__ void act_fast_x2(float x0, float x1, float& y0, float
 template <int EPI>
 __device__ __forceinline__ void act_grad_fast_x2(float x0, float x1, float& d0, float& d1) {
     if constexpr (EpiTraits<EPI>::kTanh) {
-        d0 = gelu_tanh_grad_fast(x0);
-        d1 = gelu_tanh_grad_fast(x1);
+        gelu_tanh_grad_fast_x2(x0, x1, d0, d1);
     } else {
         gelu_grad_fast_x2(x0, x1, d0, d1);
     }
