@@ -175,3 +175,24 @@ def test_activation_forms_differ_where_they_should():
     d = {k: v.cuda() for k, v in inp.items()}
     with pytest.raises(ValueError):
         binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], 2, activation="relu")
+
+
+def test_index_space_beyond_2_31_sampled():
+    """T·F > 2^31 elements (H, Y, dH of 4.3 GB each): every kernel's row,
+    column and tile offsets must be 64-bit. Ragged T and F; checked on seeded
+    token rows and hidden columns the oracle computes exactly."""
+    from tensor_transformer_mlp_block_b200 import binding
+    T, h, F, p = 65576, 64, 33032, 2
+    assert T * F > 2 ** 31
+    inp = make_shape(T, h, F, "bf16", seed_offset=23)
+    d = {k: v.cuda() for k, v in inp.items()}
+    H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p)
+    g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, p)
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == 0
+    got = dict(H=H, Y=Y, Z=Z, **g)  # stays on the GPU; only sampled slices are copied back
+    R = np.concatenate([sample_indices(T, 20, seed=1234).numpy(), [T - 1]])
+    J = np.concatenate([sample_indices(F, 40, seed=1235).numpy(), [F - 1]])
+    compare_sampled(got, inp, R, J, "bf16")
+    del H, Y, Z, g, got
+    torch.cuda.empty_cache()
