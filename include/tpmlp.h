@@ -227,7 +227,9 @@ tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t 
  * Returns the number of kinds, or -1 if a CUDA call failed.
  * tpmlp_profile_read(kind, ...) returns those totals (any out-pointer may be
  * NULL); tpmlp_profile_name(kind) its static name; tpmlp_profile_reset()
- * clears them. Not thread-safe. */
+ * clears them. The calls may come from several host threads (the state is
+ * guarded by a lock); the timing events are created on the current device,
+ * so one process times launches on one device. */
 void tpmlp_profile_enable(int on);
 int tpmlp_profile_collect(void);
 int tpmlp_profile_kinds(void);

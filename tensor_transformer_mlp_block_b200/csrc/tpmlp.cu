@@ -160,11 +160,15 @@ struct PendingRec {
     int kind;
     double flops, bytes;
 };
-bool g_prof_on = false;
+// Timing state, shared by every host thread that calls the library: the
+// flag is atomic, the records and the event pool are guarded by g_prof_mutex.
+std::atomic<bool> g_prof_on{false};
+std::mutex g_prof_mutex;
 KindTotals g_prof[K_COUNT];
 std::vector<PendingRec> g_pending;
 std::vector<cudaEvent_t> g_event_pool;
 
+// Caller holds g_prof_mutex.
 cudaEvent_t pool_event() {
     if (!g_event_pool.empty()) {
         cudaEvent_t e = g_event_pool.back();
@@ -180,12 +184,22 @@ cudaEvent_t pool_event() {
 // bracket it with two events and remember the step's algorithmic work.
 template <class Fn>
 tpmlp_status timed(int kind, double flops, double bytes, cudaStream_t st, Fn&& fn) {
-    if (!g_prof_on) return fn();
-    cudaEvent_t a = pool_event(), b = pool_event();
-    if (a == nullptr || b == nullptr) return TPMLP_ERR_CUDA;
+    if (!g_prof_on.load(std::memory_order_relaxed)) return fn();
+    cudaEvent_t a, b;
+    {
+        std::lock_guard<std::mutex> lock(g_prof_mutex);
+        a = pool_event();
+        b = pool_event();
+        if (a == nullptr || b == nullptr) {
+            if (a) g_event_pool.push_back(a);
+            if (b) g_event_pool.push_back(b);
+            return TPMLP_ERR_CUDA;
+        }
+    }
     cudaEventRecord(a, st);
     tpmlp_status s = fn();
     cudaEventRecord(b, st);
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
     g_pending.push_back({a, b, kind, flops, bytes});
     return s;
 }
@@ -1029,9 +1043,10 @@ tpmlp_status tpmlp_eval_activation(const float* x, float* y, float* dy, int64_t 
     return check_launch();
 }
 
-void tpmlp_profile_enable(int on) { g_prof_on = (on != 0); }
+void tpmlp_profile_enable(int on) { g_prof_on.store(on != 0); }
 
 int tpmlp_profile_collect(void) {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
     int rc = K_COUNT;
     for (const PendingRec& r : g_pending) {
         float ms = 0.0f;
@@ -1060,6 +1075,7 @@ const char* tpmlp_profile_name(int kind) {
 tpmlp_status tpmlp_profile_read(int kind, uint64_t* launches, double* total_ms, double* flops,
                                 double* bytes) {
     if (kind < 0 || kind >= K_COUNT) return TPMLP_ERR_INVALID;
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
     const KindTotals& t = g_prof[kind];
     if (launches) *launches = t.launches;
     if (total_ms) *total_ms = t.ms;
@@ -1069,6 +1085,7 @@ tpmlp_status tpmlp_profile_read(int kind, uint64_t* launches, double* total_ms, 
 }
 
 void tpmlp_profile_reset(void) {
+    std::lock_guard<std::mutex> lock(g_prof_mutex);
     for (KindTotals& t : g_prof) t = KindTotals{};
 }
 
