@@ -13,6 +13,9 @@
  *  - Matrices are dense, row-major, with no padding between rows.
  *  - Pointers are DEVICE pointers owned by the caller, except where a
  *    comment says otherwise. The library never allocates or frees memory.
+ *  - The pointers and `stream` belong to the device that is current on the
+ *    calling thread (cudaSetDevice); the library reads that device's
+ *    properties and launches there.
  *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
  *    stream). Work is enqueued asynchronously on it; the call returns once
  *    the launches are enqueued.
@@ -21,8 +24,10 @@
  *  - Results are deterministic: the same inputs and p give bit-identical
  *    outputs on every run.
  *  - The library keeps a small amount of process-wide state (the split
- *    policy, the wait limit, a launch counter, one device status word per
- *    device); calls from several host threads at once are not supported.
+ *    policy, the wait limit, a launch counter, per-device caches, one device
+ *    status word per device). Its caches are guarded, so host threads may
+ *    call it at the same time, each on its own stream; the settings and the
+ *    status word are shared by all of them.
  */
 #ifndef TPMLP_H
 #define TPMLP_H

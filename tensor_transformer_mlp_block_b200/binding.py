@@ -196,10 +196,11 @@ def forward(X, A, a, B, b, p: int, *, out=None, workspace=None, stream=None,
         _need(H, "H", (T, F), dt, dev)
         _need(Y, "Y", (T, F), dt, dev)
         _need(Z, "Z", (T, h), dt, dev)
-    ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
-    st = lib().tp_mlp_fwd_ex(_ptr(X), _ptr(A), _ptr(a), _ptr(B), _ptr(b), _ptr(H), _ptr(Y),
-                             _ptr(Z), T, h, F, int(p), _dtype_code(X), _act_code(activation),
-                             _ptr(ws), ws_bytes, _stream_ptr(dev, stream))
+    with torch.cuda.device(dev):
+        ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
+        st = lib().tp_mlp_fwd_ex(_ptr(X), _ptr(A), _ptr(a), _ptr(B), _ptr(b), _ptr(H), _ptr(Y),
+                                 _ptr(Z), T, h, F, int(p), _dtype_code(X), _act_code(activation),
+                                 _ptr(ws), ws_bytes, _stream_ptr(dev, stream))
     _check(st, "tp_mlp_fwd_ex")
     return H, Y, Z
 
@@ -228,11 +229,13 @@ def backward(dZ, X, A, B, H, Y, p: int, *, out=None, workspace=None, stream=None
     for name, shp, d in (("dX", (T, h), dt), ("dA", (h, F), f32), ("da", (F,), f32),
                          ("dB", (F, h), f32), ("db", (h,), f32), ("dH", (T, F), dt)):
         _need(out[name], name, shp, d, dev)
-    ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
-    st = lib().tp_mlp_bwd_ex(_ptr(dZ), _ptr(X), _ptr(A), _ptr(B), _ptr(H), _ptr(Y),
-                             _ptr(out["dX"]), _ptr(out["dA"]), _ptr(out["da"]), _ptr(out["dB"]),
-                             _ptr(out["db"]), _ptr(out["dH"]), T, h, F, int(p), _dtype_code(X),
-                             _act_code(activation), _ptr(ws), ws_bytes, _stream_ptr(dev, stream))
+    with torch.cuda.device(dev):
+        ws, ws_bytes = _workspace(T, h, F, p, dt, dev, workspace)
+        st = lib().tp_mlp_bwd_ex(_ptr(dZ), _ptr(X), _ptr(A), _ptr(B), _ptr(H), _ptr(Y),
+                                 _ptr(out["dX"]), _ptr(out["dA"]), _ptr(out["da"]),
+                                 _ptr(out["dB"]), _ptr(out["db"]), _ptr(out["dH"]), T, h, F,
+                                 int(p), _dtype_code(X), _act_code(activation), _ptr(ws), ws_bytes,
+                                 _stream_ptr(dev, stream))
     _check(st, "tp_mlp_bwd_ex")
     return out
 
@@ -250,8 +253,9 @@ def set_wait_limit_ns(ns: int) -> None:
 
 
 def last_device_status(stream=None, device=None) -> int:
-    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
-    return int(lib().tpmlp_last_device_status(_stream_ptr(dev, stream)))
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    with torch.cuda.device(dev):
+        return int(lib().tpmlp_last_device_status(_stream_ptr(dev, stream)))
 
 
 def wait_selftest(limit_ns: int, stream=None) -> None:
@@ -304,9 +308,10 @@ def eval_activation(x: torch.Tensor, form: int):
         raise ValueError("x must be a contiguous CUDA float32 tensor")
     y = torch.empty_like(x)
     dy = torch.empty_like(x)
-    _check(lib().tpmlp_eval_activation(x.data_ptr(), y.data_ptr(), dy.data_ptr(), x.numel(),
-                                       int(form), _stream_ptr(x.device, None)),
-           "tpmlp_eval_activation")
+    with torch.cuda.device(x.device):
+        _check(lib().tpmlp_eval_activation(x.data_ptr(), y.data_ptr(), dy.data_ptr(), x.numel(),
+                                           int(form), _stream_ptr(x.device, None)),
+               "tpmlp_eval_activation")
     return y, dy
 
 
@@ -338,11 +343,12 @@ def linear_forward(X, W, bias, p: int, split: str, *, out=None, workspace=None, 
         _need(bias, "bias", (N,), dt, dev)
     Y = torch.empty((T, N), dtype=dt, device=dev) if out is None else out
     _need(Y, "Y", (T, N), dt, dev)
-    n = linear_workspace_size(T, K, N, p, split, dt)
-    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
-    st = lib().tp_linear_fwd(_ptr(X), _ptr(W), _ptr(bias), _ptr(Y), T, K, N, int(p),
-                             _split_code(split), _dtype_code(X), _ptr(ws),
-                             ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
+    with torch.cuda.device(dev):
+        n = linear_workspace_size(T, K, N, p, split, dt)
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
+        st = lib().tp_linear_fwd(_ptr(X), _ptr(W), _ptr(bias), _ptr(Y), T, K, N, int(p),
+                                 _split_code(split), _dtype_code(X), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
     _check(st, "tp_linear_fwd")
     return Y
 
@@ -362,11 +368,12 @@ def linear_backward(dY, X, W, p: int, split: str, *, out=None, workspace=None, s
     _need(dX, "dX", (T, K), dt, dev)
     _need(dW, "dW", (K, N), torch.float32, dev)
     _need(db, "dbias", (N,), torch.float32, dev)
-    n = linear_workspace_size(T, K, N, p, split, dt)
-    ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
-    st = lib().tp_linear_bwd(_ptr(dY), _ptr(X), _ptr(W), _ptr(dX), _ptr(dW), _ptr(db), T, K, N,
-                             int(p), _split_code(split), _dtype_code(X), _ptr(ws),
-                             ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
+    with torch.cuda.device(dev):
+        n = linear_workspace_size(T, K, N, p, split, dt)
+        ws = torch.empty(max(n, 1), dtype=torch.uint8, device=dev) if workspace is None else workspace
+        st = lib().tp_linear_bwd(_ptr(dY), _ptr(X), _ptr(W), _ptr(dX), _ptr(dW), _ptr(db), T, K,
+                                 N, int(p), _split_code(split), _dtype_code(X), _ptr(ws),
+                                 ws.numel() * ws.element_size(), _stream_ptr(dev, stream))
     _check(st, "tp_linear_bwd")
     return dX, dW, db
 
@@ -388,10 +395,11 @@ def recompute_hidden(X, A, a, p: int, *, out=None, activation: str = "gelu", str
         H, Y = out
         _need(H, "H", (T, F), dt, dev)
         _need(Y, "Y", (T, F), dt, dev)
-    _check(lib().tp_mlp_recompute_hidden(_ptr(X), _ptr(A), _ptr(a), _ptr(H), _ptr(Y), T, h, F,
-                                         int(p), _dtype_code(X), _act_code(activation),
-                                         _stream_ptr(dev, stream)),
-           "tp_mlp_recompute_hidden")
+    with torch.cuda.device(dev):
+        _check(lib().tp_mlp_recompute_hidden(_ptr(X), _ptr(A), _ptr(a), _ptr(H), _ptr(Y), T, h, F,
+                                             int(p), _dtype_code(X), _act_code(activation),
+                                             _stream_ptr(dev, stream)),
+               "tp_mlp_recompute_hidden")
     return H, Y
 
 
@@ -401,7 +409,9 @@ def recompute_activation(H, *, out=None, activation: str = "gelu", stream=None):
         raise ValueError("H must be a contiguous CUDA tensor")
     Y = torch.empty_like(H) if out is None else out
     _need(Y, "Y", tuple(H.shape), H.dtype, H.device)
-    _check(lib().tp_mlp_recompute_activation(_ptr(H), _ptr(Y), H.numel(), _dtype_code(H),
-                                             _act_code(activation), _stream_ptr(H.device, stream)),
-           "tp_mlp_recompute_activation")
+    with torch.cuda.device(H.device):
+        _check(lib().tp_mlp_recompute_activation(_ptr(H), _ptr(Y), H.numel(), _dtype_code(H),
+                                                 _act_code(activation),
+                                                 _stream_ptr(H.device, stream)),
+               "tp_mlp_recompute_activation")
     return Y

@@ -49,8 +49,8 @@ def run_gpu(inp: dict, p: int, device="cuda:0", activation: str = "gelu"):
     d = {k: v.to(device) for k, v in inp.items()}
     H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p, activation=activation)
     g = binding.backward(d["dZ"], d["X"], d["A"], d["B"], H, Y, p, activation=activation)
-    torch.cuda.synchronize()
-    st = binding.last_device_status()
+    torch.cuda.synchronize(device)
+    st = binding.last_device_status(device=device)
     assert st == 0, f"device status {st}"
     out = dict(H=H, Y=Y, Z=Z, **g)
     return {k: v.cpu() for k, v in out.items()}

@@ -196,3 +196,16 @@ def test_index_space_beyond_2_31_sampled():
     compare_sampled(got, inp, R, J, "bf16")
     del H, Y, Z, g, got
     torch.cuda.empty_cache()
+
+
+@pytest.mark.skipif(not torch.cuda.is_available() or torch.cuda.device_count() < 2,
+                    reason="needs two GPUs")
+def test_tensors_on_a_device_other_than_the_current_one():
+    """The binding makes the tensors' device current around each call: a
+    block on cuda:1 while cuda:0 is current gives cuda:0's result."""
+    inp = make_shape(300, 200, 520, "bf16", seed_offset=31)
+    ref = run_gpu(inp, 2, device="cuda:0")
+    with torch.cuda.device(0):
+        got = run_gpu(inp, 2, device="cuda:1")
+    for k in ref:
+        assert torch.equal(ref[k], got[k]), k
