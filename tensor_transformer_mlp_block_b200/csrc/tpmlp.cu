@@ -241,7 +241,8 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
         int devn = 0;
-        cudaGetDevice(&devn);
+        if (cudaGetDevice(&devn) != cudaSuccess || devn < 0 || devn >= kMaxDevices)
+            return TPMLP_ERR_CUDA;
         if (!(g_dev[devn].attr_set & (uint64_t(1) << id))) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Cfg::SMEM_BYTES) != cudaSuccess)
@@ -282,7 +283,8 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
         int devn = 0;
-        cudaGetDevice(&devn);
+        if (cudaGetDevice(&devn) != cudaSuccess || devn < 0 || devn >= kMaxDevices)
+            return TPMLP_ERR_CUDA;
         DeviceInfo& d = g_dev[devn];
         if (!(d.attr_set_pair & (uint64_t(1) << id))) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
