@@ -191,6 +191,18 @@ tpmlp_status tpmlp_last_device_status(void* stream);
 tpmlp_status tpmlp_set_split_policy(int policy);
 int tpmlp_get_split_policy(void);
 
+/* Launch overlap (default on): the library's tensor-core and helper kernels
+ * go out as programmatic dependent launches (CUDA's
+ * cudaLaunchAttributeProgrammaticStreamSerialization). A kernel's CTAs may
+ * then start, and set up their barriers and tensor memory, on SMs its
+ * predecessor on the stream has already left; each waits for the
+ * predecessor to complete before it reads or writes global memory. Results
+ * are bit-identical with overlap on or off, and the first kernel of a call
+ * never reads the caller's data before the caller's preceding work has
+ * finished. Off: ordinary stream order. */
+void tpmlp_set_launch_overlap(int on);
+int tpmlp_get_launch_overlap(void);
+
 /* Upper bound, in nanoseconds, on any single wait inside a kernel (for data
  * from the tensor-memory accelerator, for the tensor cores, between warps).
  * Default 2e9 (2 s). A wait that runs out sets the device status word to

@@ -13,6 +13,8 @@ namespace tpmlp {
 __global__ void __launch_bounds__(256) reduce_splits_bf16_kernel(
     const float* __restrict__ ws, int splits, int64_t plane, const __nv_bfloat16* __restrict__ bias,
     __nv_bfloat16* __restrict__ out, int64_t M, int64_t N) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
     const int64_t groups = M * (N / 8);
     for (int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gi < groups;
          gi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
@@ -66,6 +68,8 @@ template <typename T, bool VEC>
 __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ X, int64_t R,
                                                             int64_t C, int64_t rows_per_chunk,
                                                             float* __restrict__ partial) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
     __shared__ float red[8][256];
     const int64_t c0 = blockIdx.x * 256 + threadIdx.x * 8;
     const int64_t r_begin = blockIdx.y * rows_per_chunk;
@@ -147,6 +151,8 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ partial,
                                                           int chunks, int64_t C,
                                                           float* __restrict__ out) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
     __shared__ float grp[8][32];
     const int64_t c = blockIdx.x * 32 + threadIdx.x;
     const int per = (chunks + 7) / 8;
@@ -246,6 +252,8 @@ __device__ __forceinline__ float4 act_f32x4(float4 v) {
 template <typename T, bool TANH, bool VEC>
 __global__ void __launch_bounds__(256, 8) recompute_act_kernel(const T* __restrict__ H,
                                                            T* __restrict__ Y, int64_t n) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
     const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
     const int64_t first = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
     if constexpr (VEC) {
@@ -296,6 +304,8 @@ __global__ void __launch_bounds__(256, 8) recompute_act_kernel(const T* __restri
 }
 
 __global__ void zero_f32_kernel(float* __restrict__ p, int64_t n) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
     for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
          i += static_cast<int64_t>(gridDim.x) * blockDim.x)
         p[i] = 0.0f;

@@ -535,6 +535,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // launched as a programmatic dependent: the prologue above overlaps the
+    // predecessor's last CTAs; its outputs are read only after this wait
+    grid_dep_wait();
+    grid_dep_launch();
 
     const int tiles = g.num_m_blocks * g.num_n_blocks;
     const int units = tiles * g.splits;

@@ -82,6 +82,19 @@ __device__ __forceinline__ void raise_timeout(volatile int* abort) {
     __threadfence_block();
 }
 
+// ------------------------------------------- programmatic dependent launch
+// With the launch attribute cudaLaunchAttributeProgrammaticStreamSerialization
+// a kernel may start before its predecessor on the stream has finished.
+// grid_dep_wait() blocks until that predecessor has completed and its memory
+// is visible; grid_dep_launch() lets the successor start once every CTA of
+// this grid has issued it or exited. Without the attribute both return at once.
+
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+__device__ __forceinline__ void grid_dep_launch() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ----------------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

@@ -39,6 +39,7 @@ constexpr int kMaxDevices = 64;
 std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_split_policy{0};
+std::atomic<bool> g_overlap{true};  // programmatic dependent launches
 
 struct DeviceInfo {
     bool init = false;
@@ -134,6 +135,35 @@ bool make_out_maps(CUtensorMap* o0, CUtensorMap* o1, const GemmArgs& g, int M, i
 
 tpmlp_status check_launch() {
     g_launches.fetch_add(1, std::memory_order_relaxed);
+    return cudaGetLastError() == cudaSuccess ? TPMLP_OK : TPMLP_ERR_CUDA;
+}
+
+// Launch a kernel that orders itself after its predecessor with
+// grid_dep_wait() before it reads any global memory. With launch overlap on
+// it goes out as a programmatic dependent launch: its CTAs take the SMs the
+// predecessor's finished CTAs leave and run their prologue (barriers, tensor
+// memory, descriptor prefetch) while the predecessor's last CTAs still run;
+// launch latency and prologue leave the critical path. Counts the launch;
+// maps errors.
+template <typename... KArgs, typename... Args>
+tpmlp_status launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = g_overlap.load(std::memory_order_relaxed) ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return TPMLP_ERR_CUDA;
+    }
     return cudaGetLastError() == cudaSuccess ? TPMLP_OK : TPMLP_ERR_CUDA;
 }
 
@@ -252,8 +282,7 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     }
     const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
     const int grid = static_cast<int>(units < dev->num_sms ? units : dev->num_sms);
-    kern<<<grid, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, tmO0, tmO1, g);
-    return check_launch();
+    return launch_dep(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1, g);
 }
 
 // Same product on CTA pairs: 256 × BN tiles, grid = 2 × (co-resident pairs).
@@ -310,8 +339,8 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     }
     const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
     const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
-    kern<<<2 * pairs, kThreads, Cfg::SMEM_BYTES, st>>>(tmA, tmB, tmO0, tmO1, g);
-    return check_launch();
+    return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
+                      g);
 }
 
 // Algorithmic bytes of one GEMM: both operands read once (bf16), the
@@ -464,15 +493,15 @@ tpmlp_status colsum_launch(const T* X, int64_t R, int64_t C, int64_t chunks, flo
                            float* out, cudaStream_t st) {
     dim3 grid(static_cast<unsigned>((C + 255) / 256), static_cast<unsigned>(chunks));
     dim3 block(32, 8);
-    if (C % 8 == 0 && aligned16(X))
-        colsum_partial_kernel<T, true><<<grid, block, 0, st>>>(X, R, C, kColsumRowsPerChunk, partial);
-    else
-        colsum_partial_kernel<T, false><<<grid, block, 0, st>>>(X, R, C, kColsumRowsPerChunk, partial);
-    tpmlp_status s = check_launch();
+    const tpmlp_status s =
+        (C % 8 == 0 && aligned16(X))
+            ? launch_dep(colsum_partial_kernel<T, true>, grid, block, 0, st, X, R, C,
+                         kColsumRowsPerChunk, partial)
+            : launch_dep(colsum_partial_kernel<T, false>, grid, block, 0, st, X, R, C,
+                         kColsumRowsPerChunk, partial);
     if (s != TPMLP_OK) return s;
-    colsum_final_kernel<<<static_cast<unsigned>((C + 31) / 32), dim3(32, 8), 0, st>>>(
-        partial, static_cast<int>(chunks), C, out);
-    return check_launch();
+    return launch_dep(colsum_final_kernel, dim3(static_cast<unsigned>((C + 31) / 32)), dim3(32, 8), 0,
+                      st, static_cast<const float*>(partial), static_cast<int>(chunks), C, out);
 }
 
 // out = 1ᵀ·X for X: R × C; algorithmic bytes = X read once + out written.
@@ -488,10 +517,9 @@ tpmlp_status reduce_splits_launch(const float* ws, int splits, int64_t M, int64_
     const int64_t groups = M * (N / 8);
     const int64_t blocks =
         clamp_grid((groups + 255) / 256, resident_blocks<reduce_splits_bf16_kernel>(256));
-    reduce_splits_bf16_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
-        ws, splits, M * N, static_cast<const __nv_bfloat16*>(bias), static_cast<__nv_bfloat16*>(out),
-        M, N);
-    return check_launch();
+    return launch_dep(reduce_splits_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
+                      ws, splits, M * N, static_cast<const __nv_bfloat16*>(bias),
+                      static_cast<__nv_bfloat16*>(out), M, N);
 }
 
 tpmlp_status reduce_splits(int kind, const float* ws, int splits, int64_t M, int64_t N,
@@ -504,20 +532,19 @@ tpmlp_status reduce_splits(int kind, const float* ws, int splits, int64_t M, int
 // takes two 8-element groups (VEC) or one element; no more blocks than the
 // device holds at once.
 template <typename T, bool TANH, bool VEC>
-void launch_recompute(const void* H, void* Y, int64_t n, cudaStream_t st) {
+tpmlp_status launch_recompute(const void* H, void* Y, int64_t n, cudaStream_t st) {
     const int64_t work = VEC ? (n / 8 + 1) / 2 : n;
     const unsigned nb = static_cast<unsigned>(
         clamp_grid((work + 255) / 256, resident_blocks<recompute_act_kernel<T, TANH, VEC>>(256)));
-    recompute_act_kernel<T, TANH, VEC>
-        <<<nb, 256, 0, st>>>(static_cast<const T*>(H), static_cast<T*>(Y), n);
+    return launch_dep(recompute_act_kernel<T, TANH, VEC>, dim3(nb), dim3(256), 0, st,
+                      static_cast<const T*>(H), static_cast<T*>(Y), n);
 }
 
 tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st) {
     if (n <= 0) return TPMLP_OK;
     return timed(K_MISC, 0.0, 4.0 * n, st, [&] {
         const int64_t blocks = clamp_grid((n + 255) / 256, resident_blocks<zero_f32_kernel>(256));
-        zero_f32_kernel<<<static_cast<unsigned>(blocks), 256, 0, st>>>(p, n);
-        return check_launch();
+        return launch_dep(zero_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p, n);
     });
 }
 
@@ -975,20 +1002,16 @@ tpmlp_status tp_mlp_recompute_activation(const void* H, void* Y, int64_t n, tpml
         using B = __nv_bfloat16;
         if (dt == TPMLP_BF16) {
             if (vec)
-                tanh_form ? launch_recompute<B, true, true>(H, Y, n, st)
-                          : launch_recompute<B, false, true>(H, Y, n, st);
-            else
-                tanh_form ? launch_recompute<B, true, false>(H, Y, n, st)
-                          : launch_recompute<B, false, false>(H, Y, n, st);
-        } else {
-            if (vec)
-                tanh_form ? launch_recompute<float, true, true>(H, Y, n, st)
-                          : launch_recompute<float, false, true>(H, Y, n, st);
-            else
-                tanh_form ? launch_recompute<float, true, false>(H, Y, n, st)
-                          : launch_recompute<float, false, false>(H, Y, n, st);
+                return tanh_form ? launch_recompute<B, true, true>(H, Y, n, st)
+                                 : launch_recompute<B, false, true>(H, Y, n, st);
+            return tanh_form ? launch_recompute<B, true, false>(H, Y, n, st)
+                             : launch_recompute<B, false, false>(H, Y, n, st);
         }
-        return check_launch();
+        if (vec)
+            return tanh_form ? launch_recompute<float, true, true>(H, Y, n, st)
+                             : launch_recompute<float, false, true>(H, Y, n, st);
+        return tanh_form ? launch_recompute<float, true, false>(H, Y, n, st)
+                         : launch_recompute<float, false, false>(H, Y, n, st);
     });
 }
 
@@ -1021,6 +1044,10 @@ tpmlp_status tpmlp_set_split_policy(int policy) {
 }
 
 int tpmlp_get_split_policy(void) { return g_split_policy.load(); }
+
+void tpmlp_set_launch_overlap(int on) { g_overlap.store(on != 0); }
+
+int tpmlp_get_launch_overlap(void) { return g_overlap.load() ? 1 : 0; }
 
 void tpmlp_set_wait_limit_ns(uint64_t ns) { g_wait_limit_ns.store(ns == 0 ? kDefaultWaitLimitNs : ns); }
 
