@@ -64,6 +64,8 @@ def _auto_policy():
     (300, 200, 520, 4, "rows"),
     (129, 64, 264, 3, "columns"),
     (1, 8, 8, 1, "rows"),
+    (64, 32, 48, 48, "columns"),     # p = N: one output column per shard
+    (64, 48, 32, 48, "rows"),        # p = K: one input row of W per shard
 ])
 def test_linear_bf16_full_oracle(T, K, N, p, split):
     inp = _inputs(T, K, N, "bf16", seed=T + K + N)

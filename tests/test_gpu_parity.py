@@ -209,3 +209,19 @@ def test_tensors_on_a_device_other_than_the_current_one():
         got = run_gpu(inp, 2, device="cuda:1")
     for k in ref:
         assert torch.equal(ref[k], got[k]), k
+
+
+@pytest.mark.parametrize("policy", [0, 2])
+@pytest.mark.parametrize("T,h,F,p", [
+    (200, 64, 64, 64),     # p = F: every shard is one hidden column
+    (200, 64, 128, 16),    # Fp = 8: shards narrower than one 64-deep k-block
+    (130, 16, 24, 24),     # tensor-core path, p = F with a ragged 24-column hidden
+    (130, 12, 20, 20),     # plain path (h, F not multiples of 8), p = F
+])
+def test_degenerate_one_column_shards(T, h, F, p, policy):
+    """The finest partitions the method allows give the unsplit result."""
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(policy)
+    inp = make_shape(T, h, F, "bf16", seed_offset=T + F + p)
+    gpu = run_gpu(inp, p)
+    compare_full(gpu, oracle_full(inp), "bf16")
