@@ -60,6 +60,9 @@ struct GemmArgs {
     const __nv_bfloat16* bias;
     const __nv_bfloat16* aux;
     uint64_t wait_limit_ns;
+    // GeLU′ epilogues: if set, column sums of the stored (bf16) output over
+    // each 32-row block go to colsum_out[(row / 32)·N + col] (fp32)
+    float* colsum_out;
 };
 
 constexpr int kBM = 128;
@@ -260,6 +263,25 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return *reinterpret_cast<uint32_t*>(&v);
 }
 
+// Column sums of a 32 × 32 block held one row per lane (x[j] = column j of
+// this lane's row): lane l returns the sum of column l over the 32 rows. Five
+// exchange rounds; in each, a lane keeps half of its remaining columns and
+// adds its partner's values of them, so the adds follow a fixed pairwise tree
+// over the rows and the result is the same on every run.
+__device__ __forceinline__ float warp_column_sums32(float (&x)[32], int lane) {
+#pragma unroll
+    for (int w = 16; w >= 1; w >>= 1) {
+        const bool upper = (lane & w) != 0;
+#pragma unroll
+        for (int i = 0; i < w; ++i) {
+            const float send = upper ? x[i] : x[i + w];
+            const float keep = upper ? x[i + w] : x[i];
+            x[i] = keep + __shfl_xor_sync(0xffffffffu, send, w);
+        }
+    }
+    return x[0];
+}
+
 __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
     const __nv_bfloat162* p = reinterpret_cast<const __nv_bfloat162*>(&v);
 #pragma unroll
@@ -356,6 +378,18 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             tma_store_3d(tmO0, slot, col0, row0, 0);
             if constexpr (EpiTraits<EPI>::kAct) tma_store_3d(tmO1, slot + 2048, col0, row0, 0);
             bulk_commit();
+        }
+        if constexpr (EpiTraits<EPI>::kDAct) {
+            // da's partial over this chunk's 32 rows, from the values just stored
+            // (rows beyond M and columns beyond N hold zeros)
+            if (g.colsum_out != nullptr) {
+                float x[32];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) unpack_bf16x8(o0[q], x + 8 * q);
+                const float s = warp_column_sums32(x, lane);
+                if (row0 < g.M && col0 + lane < g.N)
+                    g.colsum_out[static_cast<int64_t>(row0 >> 5) * g.N + col0 + lane] = s;
+            }
         }
     }
 }

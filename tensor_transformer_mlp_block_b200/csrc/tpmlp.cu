@@ -370,12 +370,18 @@ tpmlp_status gemm_tc_pick(const void* Aop, const void* Bop, int M, int N, int K,
     return gemm_tc_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, splits, g, st);
 }
 
+// Shortest K loop per work unit for which the relaying epilogue pays
+// (measured on the 7B-class and GPT-2-class shapes).
+constexpr int kRelayMinKAct = 3072;    // GeLU and GeLU′ epilogues
+constexpr int kRelayMinKPlain = 2048;  // bias and fp32 epilogues
+
 template <int BN, bool A_MN, bool B_MN, int EPI>
 tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K, int splits,
                      GemmArgs g, cudaStream_t st) {
     return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K, splits), st, [&] {
         const int k_per_unit = splits > 1 ? K / splits : K;
-        const int threshold = (EpiTraits<EPI>::kAct || EpiTraits<EPI>::kDAct) ? 3072 : 2048;
+        const int threshold =
+            (EpiTraits<EPI>::kAct || EpiTraits<EPI>::kDAct) ? kRelayMinKAct : kRelayMinKPlain;
         if (k_per_unit < threshold)
             return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, splits, g, st);
         return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, splits, g, st);
@@ -404,6 +410,9 @@ struct Plan {
 };
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// Partial rows of da written by the GeLU′ epilogue (32 token rows each).
+int64_t da_partial_rows(int64_t T) { return T > 0 ? (T + 31) / 32 : 1; }
 
 // Shard groups S for the two row-parallel products (M = T, N = h, K = F).
 // S = 1 runs each output tile's K loop through all p shards in TMEM; S > 1
@@ -457,7 +466,9 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
     pl->off_cs_h = off;
     off += round256(static_cast<size_t>(pl->chunks) * h * sizeof(float));
     pl->off_cs_f = off;
-    off += round256(static_cast<size_t>(pl->chunks) * F * sizeof(float));
+    // tensor-core path: da's partials come from the GeLU′ epilogue, one row per
+    // 32 token rows; plain path: the column-sum kernel's 128-row chunks
+    off += round256(static_cast<size_t>(pl->tc ? da_partial_rows(T) : pl->chunks) * F * sizeof(float));
     pl->total = off;
     return true;
 }
@@ -510,6 +521,16 @@ tpmlp_status colsum(int kind, const T* X, int64_t R, int64_t C, int64_t chunks, 
                     float* out, cudaStream_t st) {
     return timed(kind, 0.0, sizeof(T) * double(R) * C + 4.0 * C, st,
                  [&] { return colsum_launch(X, R, C, chunks, partial, out, st); });
+}
+
+// Pass 2 alone: out[c] = Σ over `rows` partial rows of partial[r][c], in
+// ascending r (partials written by a GEMM epilogue).
+tpmlp_status colsum_finish(int kind, const float* partial, int64_t rows, int64_t C, float* out,
+                           cudaStream_t st) {
+    return timed(kind, 0.0, 4.0 * double(rows) * C + 4.0 * C, st, [&] {
+        return launch_dep(colsum_final_kernel, dim3(static_cast<unsigned>((C + 31) / 32)),
+                          dim3(32, 8), 0, st, partial, static_cast<int>(rows), C, out);
+    });
 }
 
 tpmlp_status reduce_splits_launch(const float* ws, int splits, int64_t M, int64_t N,
@@ -812,13 +833,23 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // db = 1ᵀ·dZ
         TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
+        // With the relaying epilogue (long K) the math warps have room to also
+        // leave the column sums of dH over each 32-row block in cs_f
+        // (ceil(T/32) rows of F); da then needs only their ordered sum. With
+        // short K the extra epilogue work costs more than the separate pass.
+        const bool fused_da = h >= kRelayMinKAct;
         GemmArgs g2{};
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
+        g2.colsum_out = fused_da ? cs_f : nullptr;
         TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
         // da = 1ᵀ·dH
-        TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
+        if (fused_da)
+            TPMLP_TRY(colsum_finish(K_B2_DA, cs_f, da_partial_rows(T), F, da, st));
+        else
+            TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f,
+                             da, st));
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
         GemmArgs g3{};
         g3.out0 = dB;

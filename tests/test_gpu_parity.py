@@ -38,6 +38,8 @@ def test_tiny_fp32_full():
     (129, 64, 264, 3),     # one row past a tile, single k-block, Fp = 88
     (1, 8, 8, 1),          # single token, smallest aligned shape
     (640, 96, 776, 1),     # p = 1: the unsplit MLP
+    (300, 3072, 520, 2),   # h ≥ 3072: relaying epilogues, da summed in the GeLU′ epilogue
+    (100, 3072, 264, 3),   # the same on the one-CTA kernel (T ≤ 128), ragged F
 ])
 def test_bf16_full_oracle(T, h, F, p):
     inp = make_shape(T, h, F, "bf16", seed_offset=T + h + F)
