@@ -46,7 +46,9 @@ def parse_args(argv=None):
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default="7b")
-    ap.add_argument("--e2e-steps", type=int, default=30)
+    ap.add_argument("--e2e-steps", type=int, default=None,
+                    help="steps of the end-to-end measurement (default: --steps, so that both "
+                         "numbers cover the same sustained power-capped interval)")
     ap.add_argument("--graph", action="store_true",
                     help="capture one step in a CUDA graph and time its replays")
     ap.add_argument("--activation", choices=["gelu", "gelu_tanh"], default="gelu",
@@ -64,6 +66,8 @@ def parse_args(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
                     help="target seconds of oracle work for the CPU baseline sample")
     args = ap.parse_args(argv)
+    if args.e2e_steps is None:
+        args.e2e_steps = args.steps
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     return args
