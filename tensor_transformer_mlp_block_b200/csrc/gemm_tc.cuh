@@ -60,8 +60,9 @@ struct GemmArgs {
     const __nv_bfloat16* bias;
     const __nv_bfloat16* aux;
     uint64_t wait_limit_ns;
-    // GeLU′ epilogues: if set, column sums of the stored (bf16) output over
-    // each 32-row block go to colsum_out[(row / 32)·N + col] (fp32)
+    // GeLU′ epilogues with the relay: if set, column sums of the stored (bf16)
+    // output go to colsum_out[r·N + col] (fp32), one row r per 64 rows a
+    // computing warp handles in a 128-row CTA tile (see epilogue_role)
     float* colsum_out;
 };
 
@@ -302,10 +303,14 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
 // columns outside the output. The slot is reused only after the previous
 // store of this warp has finished reading it.
 template <int EPI>
+// cs_mode (GeLU′ epilogues with colsum_out): 0 = none; 1 = keep this chunk's
+// stored values in csx; 2 = add them to csx, reduce csx over the 32 lanes
+// and write the column sums to colsum_out row cs_row (if cs_row ≥ 0).
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensorMap* tmO0,
                                                const CUtensorMap* tmO1, const uint32_t (&acc)[32],
                                                int row0, int col0, int split, uint32_t slot,
-                                               int lane) {
+                                               int lane, float (&csx)[32], int cs_mode,
+                                               int64_t cs_row) {
     const int row = row0 + lane;
     const bool any = (row0 < g.M) && (col0 < g.N);
     if constexpr (EPI == EPI_F32) {
@@ -380,15 +385,21 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             bulk_commit();
         }
         if constexpr (EpiTraits<EPI>::kDAct) {
-            // da's partial over this chunk's 32 rows, from the values just stored
-            // (rows beyond M and columns beyond N hold zeros)
-            if (g.colsum_out != nullptr) {
-                float x[32];
+            // da's partial from the values just stored (rows beyond M and
+            // columns beyond N hold zeros): this lane's row of the chunk, then
+            // with cs_mode 2 the sum over both chunks' 64 rows per column
+            if (cs_mode != 0) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) unpack_bf16x8(o0[q], x + 8 * q);
-                const float s = warp_column_sums32(x, lane);
-                if (row0 < g.M && col0 + lane < g.N)
-                    g.colsum_out[static_cast<int64_t>(row0 >> 5) * g.N + col0 + lane] = s;
+                for (int q = 0; q < 4; ++q) {
+                    float x[8];
+                    unpack_bf16x8(o0[q], x);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) csx[8 * q + i] = cs_mode == 1 ? x[i] : csx[8 * q + i] + x[i];
+                }
+                if (cs_mode == 2) {
+                    const float s = warp_column_sums32(csx, lane);
+                    if (cs_row >= 0 && col0 + lane < g.N) g.colsum_out[cs_row * g.N + col0 + lane] = s;
+                }
             }
         }
     }
@@ -450,6 +461,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                static_cast<uint32_t>(buf * BN);
         bool failed = false;
+        float csx[32];  // da partial of the current columns (relay, GeLU′ only)
 #pragma unroll 1
         for (int i = 0; i < kChunks; ++i) {
             const int c = half * kChunks + i;
@@ -483,7 +495,13 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 ++xcount;
                 continue;
             }
-            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, split, slot, lane);
+            // da partials (relay only): the own rows and the partner's rows of these
+            // columns form one row of colsum_out per computing warp and CTA tile
+            const bool cs_on = RELAY && g.colsum_out != nullptr;
+            const int64_t cs_row =
+                tile_row0 < g.M ? static_cast<int64_t>(tile_row0 / kBM) * 2 + (quad - 2) : -1;
+            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, split, slot, lane,
+                                csx, cs_on ? 1 : 0, cs_row);
             if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
                 const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
@@ -503,7 +521,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 mbar_arrive(smem_u32(&xempty[pair_id]));
                 ++xcount;
                 epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, split,
-                                    slot, lane);
+                                    slot, lane, csx, cs_on ? 2 : 0, cs_row);
             }
         }
         if (failed) {

@@ -12,7 +12,9 @@
 //                        are added in ascending order before the bias
 // and the backward four GEMMs plus two column sums (chain rule):
 //   B2  dH = (dZ·Bᵀ) ⊙ GeLU′(H)   B3  dB = Yᵀ·dZ   B4  dA = Xᵀ·dH
-//   B5  dX = Σ_i dH_i·A_iᵀ (ordered shard sum, as F2)   db, da column sums.
+//   B5  dX = Σ_i dH_i·A_iᵀ (ordered shard sum, as F2)   db, da column sums
+// (for long K the B2 epilogue itself writes da's per-32-row partials, and
+// only their ordered sum remains).
 #include <cuda.h>
 #include <cuda_runtime.h>
 
@@ -411,8 +413,9 @@ struct Plan {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// Partial rows of da written by the GeLU′ epilogue (32 token rows each).
-int64_t da_partial_rows(int64_t T) { return T > 0 ? (T + 31) / 32 : 1; }
+// Partial rows of da written by the relaying GeLU′ epilogue: two per 128-row
+// CTA tile (one per computing warp, 64 rows each).
+int64_t da_partial_rows(int64_t T) { return T > 0 ? 2 * ((T + kBM - 1) / kBM) : 1; }
 
 // Shard groups S for the two row-parallel products (M = T, N = h, K = F).
 // S = 1 runs each output tile's K loop through all p shards in TMEM; S > 1
@@ -466,8 +469,9 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
     pl->off_cs_h = off;
     off += round256(static_cast<size_t>(pl->chunks) * h * sizeof(float));
     pl->off_cs_f = off;
-    // tensor-core path: da's partials come from the GeLU′ epilogue, one row per
-    // 32 token rows; plain path: the column-sum kernel's 128-row chunks
+    // tensor-core path: da's partials come from the GeLU′ epilogue (two rows per
+    // 128 token rows) or from the column-sum kernel (one per 128); plain path:
+    // the column-sum kernel
     off += round256(static_cast<size_t>(pl->tc ? da_partial_rows(T) : pl->chunks) * F * sizeof(float));
     pl->total = off;
     return true;
@@ -833,10 +837,10 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // db = 1ᵀ·dZ
         TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
-        // With the relaying epilogue (long K) the math warps have room to also
-        // leave the column sums of dH over each 32-row block in cs_f
-        // (ceil(T/32) rows of F); da then needs only their ordered sum. With
-        // short K the extra epilogue work costs more than the separate pass.
+        // With the relaying epilogue (long K) the computing warps have room to
+        // also leave the column sums of dH in cs_f (two partial rows per
+        // 128-row tile); da then needs only their ordered sum. With short K
+        // the extra epilogue work costs more than the separate pass.
         const bool fused_da = h >= kRelayMinKAct;
         GemmArgs g2{};
         g2.out0 = dH;
