@@ -227,3 +227,14 @@ def test_degenerate_one_column_shards(T, h, F, p, policy):
     inp = make_shape(T, h, F, "bf16", seed_offset=T + F + p)
     gpu = run_gpu(inp, p)
     compare_full(gpu, oracle_full(inp), "bf16")
+
+
+@pytest.mark.parametrize("T", [64, 129, 257, 385])
+def test_fused_da_partials_at_tile_edges(T):
+    """da summed in the relaying GeLU′ epilogue (h ≥ 3072) when CTA tiles are
+    partly or wholly past the last token row: T = 64 (one CTA, the computing
+    warps' own rows all past T), 129 and 385 (the pair's second CTA holds one
+    valid row), 257."""
+    inp = make_shape(T, 3072, 264, "bf16", seed_offset=T + 71)
+    gpu = run_gpu(inp, 2)
+    compare_full(gpu, oracle_full(inp), "bf16")
