@@ -21,19 +21,56 @@ TOL = {"bf16": 2e-2, "fp32": 1e-5}
 STORED = ("H", "Y", "dH")
 UNIT_ROUNDOFF = {"bf16": 2.0 ** -8, "fp32": 2.0 ** -24}
 
+# The products that consume a stored bf16 activation (Z = Y·B, dX = dH·Aᵀ,
+# dA = Xᵀ·dH, dB = Yᵀ·dZ, da = 1ᵀ·dH) inherit its rounding: an element
+# Σ_k a_k·b_k whose a_k each carry a relative error ≤ 2⁻⁹ is off by at most
+# 2⁻⁹·Σ_k |a_k·b_k| ≤ u·(Σ_k (a_k·b_k)²)^½ for up to 4 terms (Cauchy–Schwarz),
+# and for more terms that is still above 3σ of the random rounding errors.
+# With many terms it is far below tol·rms; with 1–2 tokens an element of dA
+# or dB is a single product, where the rms-relative bound alone does not hold.
+# That allowance is added element by element, as for the stored activations.
+
+
+class OracleResult(dict):
+    """The oracle's outputs, with the rounded inputs they were computed from."""
+
+    inputs: dict
+
+
+def product_allowance(key: str, ref: OracleResult, dtype: str):
+    """u·(Σ_k (a_k·b_k)²)^½ for the products that read a stored bf16
+    activation, element by element (None for the others, or for fp32)."""
+    if dtype != "bf16" or not hasattr(ref, "inputs"):
+        return None
+    n = ref.inputs
+    u = UNIT_ROUNDOFF["bf16"]
+    Y, dH = ref["Y"], ref["dH"]
+    if key == "Z":
+        return u * np.sqrt((Y * Y) @ (n["B"] * n["B"]))
+    if key == "dX":
+        return u * np.sqrt((dH * dH) @ (n["A"] * n["A"]).T)
+    if key == "dA":
+        return u * np.sqrt((n["X"] * n["X"]).T @ (dH * dH))
+    if key == "dB":
+        return u * np.sqrt((Y * Y).T @ (n["dZ"] * n["dZ"]))
+    if key == "da":
+        return u * np.sqrt((dH * dH).sum(axis=0))
+    return None
+
 
 def to_np(t: torch.Tensor) -> np.ndarray:
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def rel_err(got, ref, u: float = 0.0) -> float:
-    """max over elements of (|got − ref| − u·|ref|), divided by rms(ref)."""
+def rel_err(got, ref, u: float = 0.0, allow=None) -> float:
+    """max over elements of (|got − ref| − u·|ref| − allow), divided by rms(ref)."""
     got = np.asarray(got, dtype=np.float64)
     ref = np.asarray(ref, dtype=np.float64)
     if ref.size == 0:
         return 0.0
     rms = float(np.sqrt(np.mean(ref * ref)))
-    err = float(np.max(np.abs(got - ref) - u * np.abs(ref)))
+    slack = u * np.abs(ref) + (0.0 if allow is None else np.asarray(allow, dtype=np.float64))
+    err = float(np.max(np.abs(got - ref) - slack))
     if rms == 0.0:
         return max(err, 0.0)
     return err / rms
@@ -61,14 +98,16 @@ def oracle_full(inp: dict, act: int = 0):
     n = {k: to_np(v) for k, v in inp.items()}
     H, Y, Z = oracle.forward(n["X"], n["A"], n["a"], n["B"], n["b"], act)
     g = oracle.backward(n["X"], n["A"], n["B"], H, Y, n["dZ"], act)
-    return dict(H=H, Y=Y, Z=Z, **g)
+    out = OracleResult(H=H, Y=Y, Z=Z, **g)
+    out.inputs = n
+    return out
 
 
 def compare_full(gpu: dict, ref: dict, dtype: str, keys=None) -> dict:
     tol = TOL[dtype]
     errs = {}
     for k in keys or ref:
-        errs[k] = rel_err(to_np(gpu[k]), ref[k], _u(k, dtype))
+        errs[k] = rel_err(to_np(gpu[k]), ref[k], _u(k, dtype), product_allowance(k, ref, dtype))
     bad = {k: e for k, e in errs.items() if not e <= tol}
     assert not bad, f"outside {tol}·rms: {bad} (all: {errs})"
     print("parity", {k: round(v, 5) for k, v in errs.items()})

@@ -1,0 +1,47 @@
+"""A seeded sweep of random shapes through the whole block against the full
+oracle: token counts from 1 to ~700 (ragged against every tile size),
+hidden and shard sizes on both sides of the tensor-core path's 16-byte rule,
+p from 1 to 8, both split policies, both activations, launch overlap on and
+off. The shapes come from a fixed seed, so the sweep is the same every run."""
+import random
+
+import pytest
+
+from parity_util import compare_full, oracle_full, run_gpu
+from tensor_transformer_mlp_block_b200 import binding
+from tensor_transformer_mlp_block_b200.inputs import make_shape
+
+pytestmark = pytest.mark.gpu
+
+
+def _cases(n=48, seed=2024):
+    rng = random.Random(seed)
+    out = []
+    for i in range(n):
+        p = rng.choice([1, 2, 3, 4, 8])
+        if i % 6 == 5:  # plain path: h or F not a multiple of 8
+            h = rng.choice([4, 12, 20, 36])
+            Fp = rng.choice([3, 5, 6, 10])
+        else:           # tensor-core path
+            h = 8 * rng.randint(1, 48)
+            Fp = 8 * rng.randint(1, 40)
+        T = rng.choice([1, 2, 17, 64, 127, 128, 129, 255, 256, 257]) if i % 3 == 0 else rng.randint(1, 700)
+        out.append(dict(T=T, h=h, F=Fp * p, p=p, policy=rng.choice([0, 1, 2]),
+                        act=rng.choice(["gelu", "gelu_tanh"]), overlap=rng.random() < 0.7, seed=i))
+    return out
+
+
+@pytest.fixture(autouse=True)
+def _restore():
+    yield
+    binding.set_split_policy(0)
+    binding.set_launch_overlap(True)
+
+
+@pytest.mark.parametrize("c", _cases(), ids=lambda c: "T{T}-h{h}-F{F}-p{p}-s{policy}-{act}-o{overlap:d}".format(**c))
+def test_random_shape_against_oracle(c):
+    binding.set_split_policy(c["policy"])
+    binding.set_launch_overlap(c["overlap"])
+    inp = make_shape(c["T"], c["h"], c["F"], "bf16", seed_offset=1000 + c["seed"])
+    gpu = run_gpu(inp, c["p"], activation=c["act"])
+    compare_full(gpu, oracle_full(inp, act=1 if c["act"] == "gelu_tanh" else 0), "bf16")
