@@ -45,3 +45,49 @@ def test_random_shape_against_oracle(c):
     inp = make_shape(c["T"], c["h"], c["F"], "bf16", seed_offset=1000 + c["seed"])
     gpu = run_gpu(inp, c["p"], activation=c["act"])
     compare_full(gpu, oracle_full(inp, act=1 if c["act"] == "gelu_tanh" else 0), "bf16")
+
+
+def _linear_cases(n=24, seed=77):
+    rng = random.Random(seed)
+    out = []
+    for i in range(n):
+        p = rng.choice([1, 2, 3, 4, 8])
+        split = rng.choice(["columns", "rows"])
+        if i % 6 == 5:  # plain path
+            K = rng.choice([4, 12, 20]) * (p if split == "rows" else 1)
+            N = rng.choice([6, 10, 14]) * (p if split == "columns" else 1)
+        else:
+            K = 8 * rng.randint(1, 40) * (p if split == "rows" else 1)
+            N = 8 * rng.randint(1, 40) * (p if split == "columns" else 1)
+        T = rng.choice([1, 2, 127, 128, 129, 256, 257]) if i % 3 == 0 else rng.randint(1, 600)
+        out.append(dict(T=T, K=K, N=N, p=p, split=split, policy=rng.choice([0, 1, 2]),
+                        overlap=rng.random() < 0.7, seed=i))
+    return out
+
+
+@pytest.mark.parametrize("c", _linear_cases(),
+                         ids=lambda c: "T{T}-K{K}-N{N}-p{p}-{split}-s{policy}-o{overlap:d}".format(**c))
+def test_random_linear_against_oracle(c):
+    import numpy as np
+    import torch
+
+    import oracle
+    from parity_util import TOL, rel_err, to_np
+    binding.set_split_policy(c["policy"])
+    binding.set_launch_overlap(c["overlap"])
+    g = torch.Generator().manual_seed(500 + c["seed"])
+    T, K, N = c["T"], c["K"], c["N"]
+    X = torch.randn((T, K), generator=g).to(torch.bfloat16)
+    W = (torch.randn((K, N), generator=g) / np.sqrt(K)).to(torch.bfloat16)
+    bias = (torch.randn((N,), generator=g) * 0.1).to(torch.bfloat16)
+    dY = torch.randn((T, N), generator=g).to(torch.bfloat16)
+    Y = binding.linear_forward(X.cuda(), W.cuda(), bias.cuda(), c["p"], c["split"])
+    dX, dW, db = binding.linear_backward(dY.cuda(), X.cuda(), W.cuda(), c["p"], c["split"])
+    torch.cuda.synchronize()
+    assert binding.last_device_status() == binding.OK
+    n = dict(X=to_np(X), W=to_np(W), bias=to_np(bias), dY=to_np(dY))
+    ref_Y = oracle.linear_forward(n["X"], n["W"], n["bias"])
+    ref_dX, ref_dW, ref_db = oracle.linear_backward(n["X"], n["W"], n["dY"])
+    errs = {"Y": rel_err(to_np(Y.cpu()), ref_Y), "dX": rel_err(to_np(dX.cpu()), ref_dX),
+            "dW": rel_err(to_np(dW.cpu()), ref_dW), "db": rel_err(to_np(db.cpu()), ref_db)}
+    assert all(e <= TOL["bf16"] for e in errs.values()), errs
