@@ -91,3 +91,24 @@ def test_random_linear_against_oracle(c):
     errs = {"Y": rel_err(to_np(Y.cpu()), ref_Y), "dX": rel_err(to_np(dX.cpu()), ref_dX),
             "dW": rel_err(to_np(dW.cpu()), ref_dW), "db": rel_err(to_np(db.cpu()), ref_db)}
     assert all(e <= TOL["bf16"] for e in errs.values()), errs
+
+
+def _fp32_cases(n=12, seed=5):
+    rng = random.Random(seed)
+    out = []
+    for i in range(n):
+        p = rng.choice([1, 2, 3, 4])
+        out.append(dict(T=rng.choice([1, 2, 15, 16, 17, 100, 257, 513]), h=rng.randint(1, 40),
+                        F=rng.randint(1, 24) * p, p=p, act=rng.choice(["gelu", "gelu_tanh"]),
+                        overlap=rng.random() < 0.7, seed=i))
+    return out
+
+
+@pytest.mark.parametrize("c", _fp32_cases(),
+                         ids=lambda c: "T{T}-h{h}-F{F}-p{p}-{act}-o{overlap:d}".format(**c))
+def test_random_fp32_shape_against_oracle(c):
+    """fp32 (plain FFMA kernels, no TF32): within 1e-5·rms of the oracle."""
+    binding.set_launch_overlap(c["overlap"])
+    inp = make_shape(c["T"], c["h"], c["F"], "fp32", seed_offset=3000 + c["seed"])
+    gpu = run_gpu(inp, c["p"], activation=c["act"])
+    compare_full(gpu, oracle_full(inp, act=1 if c["act"] == "gelu_tanh" else 0), "fp32")
