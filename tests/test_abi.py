@@ -100,6 +100,35 @@ def test_workspace_size_host_logic(lib):
         binding.set_split_policy(3)
 
 
+def _r256(x):
+    return (x + 255) // 256 * 256
+
+
+def test_workspace_size_formula(lib):
+    """The workspace holds, each part rounded up to 256 bytes: the fp32 shard
+    partials S·T·h when the row products are split by shard, db's column-sum
+    partials ⌈T/128⌉·h, and da's: 2·⌈T/128⌉·F on the tensor-core path (two per
+    128-row tile when the GeLU′ epilogue sums them), ⌈T/128⌉·F on the plain path."""
+    import torch
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(1)
+    try:
+        for T, h, F, p in [(8192, 4096, 16384, 2), (300, 200, 520, 2), (1, 8, 8, 1), (129, 64, 264, 3)]:
+            c = -(-T // 128)
+            assert binding.workspace_size(T, h, F, p) == _r256(4 * c * h) + _r256(4 * 2 * c * F), (T, h, F)
+        assert binding.workspace_size(37, 12, 44, 2) == _r256(4 * 12) + _r256(4 * 44)  # plain path
+        assert binding.workspace_size(512, 12, 48, 2, torch.float32) == _r256(16 * 12) + _r256(16 * 48)
+        assert binding.workspace_size(0, 12, 44, 2) == _r256(4 * 12) + _r256(4 * 44)
+        # the 7B-class step: 9 MiB
+        assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20
+        binding.set_split_policy(2)  # split by shard: p planes of T·h fp32 in front
+        T, h, F, p = 384, 320, 1024, 4
+        assert binding.workspace_size(T, h, F, p) == (_r256(4 * p * T * h) + _r256(4 * 3 * h)
+                                                      + _r256(4 * 6 * F))
+    finally:
+        binding.set_split_policy(0)
+
+
 def test_product_path_refuses_cpu_tensors():
     import torch
     from tensor_transformer_mlp_block_b200 import binding
