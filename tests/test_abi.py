@@ -129,6 +129,25 @@ def test_workspace_size_formula(lib):
         binding.set_split_policy(0)
 
 
+def test_automatic_split_plan_for_the_named_workloads(lib):
+    """The automatic policy keeps the row products unsplit when the output
+    tiles fill the GPU (7B: 32 × 16 pair tiles over 74 pairs; GPT-2, 350M) and
+    splits them by shard when they do not (175B: 8 × 48 pair tiles over 74
+    pairs -> 2 shard groups). Seen through the workspace, which holds the
+    split planes. (Without a GPU the planner assumes 148 SMs.)"""
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(0)
+
+    def planes(T, h, F, p):
+        c = -(-T // 128)
+        extra = binding.workspace_size(T, h, F, p) - _r256(4 * c * h) - _r256(8 * c * F)
+        return extra / (4 * T * h)
+    assert planes(8192, 4096, 16384, 2) == 0
+    assert planes(4096, 768, 3072, 2) == 0
+    assert planes(6144, 1024, 4096, 4) == 0
+    assert planes(2048, 12288, 49152, 8) == 2
+
+
 def test_product_path_refuses_cpu_tensors():
     import torch
     from tensor_transformer_mlp_block_b200 import binding
