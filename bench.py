@@ -35,7 +35,12 @@ sys.path.insert(0, ROOT)
 METRIC = "TP-MLP fwd+bwd TFLOP/s (bf16, 1 B200) and % of dense BF16 tensor peak"
 UNIT = "TFLOP/s"
 DATASHEET_BF16_DENSE_TFLOPS = 2250.0  # NVIDIA B200 datasheet (HGX B200), dense BF16
-FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# Used only when the measured peaks of this machine are absent: an earlier
+# measurement on the same kind of B200 (copy bandwidth, cuBLAS bf16 burst).
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+# A timed region at least this long under an active power cap runs in the
+# sustained regime; shorter regions run at burst clocks.
+SUSTAINED_MIN_SECONDS = 1.0
 L2_BYTES = 126 * 1024 * 1024
 
 
@@ -45,7 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--config", default="7b")
+    ap.add_argument("--config", default="175b",
+                    help="workload preset (default: the largest, 175b; also 7b, 350m, gpt2-small, tiny)")
     ap.add_argument("--e2e-steps", type=int, default=None,
                     help="steps of the end-to-end measurement (default: --steps, so that both "
                          "numbers cover the same sustained power-capped interval)")
@@ -61,6 +67,10 @@ def parse_args(argv=None):
     ap.add_argument("--block", choices=["mlp", "attn-proj"], default="mlp",
                     help="mlp: the MLP block (default); attn-proj: the attention layer's "
                          "tensor-parallel projections (QKV split by columns, output by rows)")
+    ap.add_argument("--split-policy", type=int, choices=[0, 1, 2, 3], default=0,
+                    help="work schedule of the products (tpmlp_set_split_policy): 0 automatic "
+                         "(default), 1 whole tiles only, 2 one unit per shard for the row "
+                         "products, 3 stream-K tail wherever valid")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle CPU baseline (for profiler runs)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0,
@@ -127,13 +137,30 @@ def aggregate(flops_per_step_per_rank: float, steps: int, max_seconds: float, wo
 # ------------------------------------------------------------------- peaks
 
 def load_peaks():
+    """This machine's measured peaks (copy bandwidth, bf16 GEMM burst and, if
+    recorded, sustained), else the fallback figures (no sustained one)."""
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
         with open(path) as f:
             p = json.load(f)
-        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+        out = {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops")}
+        if p.get("bf16_tflops_sustained") is not None:
+            out["bf16_tflops_sustained"] = float(p["bf16_tflops_sustained"])
+        return out, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def pick_tensor_peak(peaks: dict, src: str, region_s: float, clocks: dict):
+    """The bf16 peak that matches the regime of the timed region: the
+    sustained figure only for a region of SUSTAINED_MIN_SECONDS or more in
+    which the power cap was active, the burst figure otherwise."""
+    capped = "sw_power_cap" in (clocks.get("reasons") or [])
+    if region_s >= SUSTAINED_MIN_SECONDS and capped and "bf16_tflops_sustained" in peaks:
+        return peaks["bf16_tflops_sustained"], (
+            f"{src} bf16 sustained: timed region {region_s:.2f} s under sw_power_cap")
+    why = "short" if region_s < SUSTAINED_MIN_SECONDS else "not power-capped"
+    return peaks["bf16_tflops"], f"{src} bf16 burst: timed region {region_s:.2f} s ({why})"
 
 
 def source_hash() -> str:
@@ -286,6 +313,7 @@ def bench_ours(args, cfg, world, rank, local):
     gout = dict(dX=torch.empty((T, h), dtype=dt, device=dev), dA=torch.empty((h, F), dtype=f32, device=dev),
                 da=torch.empty((F,), dtype=f32, device=dev), dB=torch.empty((F, h), dtype=f32, device=dev),
                 db=torch.empty((h,), dtype=f32, device=dev), dH=torch.empty((T, F), dtype=dt, device=dev))
+    binding.set_split_policy(args.split_policy)  # the workspace size depends on it
     ws = torch.empty(max(binding.workspace_size(T, h, F, p, dt), 1), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
     binding.set_launch_overlap(args.launch_overlap == "on")
@@ -402,24 +430,45 @@ def bench_ours(args, cfg, world, rank, local):
     max_seconds = max_over_ranks(seconds, dev)
     agg = aggregate(flops_per_step, args.steps, max_seconds, world)
 
-    # dominant kernel and its roofline (tensor-bound: algorithmic flops / event time)
+    # Per-kernel times inside the step. The event pass brackets every launch
+    # with an event pair, which stops the launch overlap between neighbours,
+    # so its durations add up to a little more than the step. Each kernel's
+    # in-step time is its event time scaled by (step time / sum of the event
+    # times of one step): the shares come from the events, the total from the
+    # timed region itself, and the in-step times add up to the step.
+    step_ms = 1e3 * seconds / args.steps
+    event_step_ms = sum(v["ms"] for v in kinds.values()) / kernel_pass_steps
+    scale = step_ms / event_step_ms if event_step_ms > 0 else 1.0
+    per_kernel = {}
+    for k, v in kinds.items():
+        ev_ms = v["ms"] / v["launches"]
+        in_ms = ev_ms * scale
+        per_kernel[k] = {"launches_per_step": v["launches"] / kernel_pass_steps,
+                         "ms_per_launch": in_ms, "event_ms_per_launch": ev_ms,
+                         "tflops": (v["flops"] / v["launches"] / in_ms / 1e9) if v["flops"] else None,
+                         "gbs": v["bytes"] / v["launches"] / in_ms / 1e6}
+
+    # dominant kernel and its roofline (tensor-bound: algorithmic flops / in-step time)
+    tensor_peak, peak_source = pick_tensor_peak(peaks, peaks_src, seconds, clocks)
     top_name, top = max(kinds.items(), key=lambda kv: kv[1]["ms"])
-    per_launch_ms = top["ms"] / top["launches"]
-    achieved = top["flops"] / top["launches"] / (per_launch_ms / 1e3) / 1e12
-    peak = peaks["bf16_tflops_sustained"]
-    roofline = {"bound": "tensor", "kernel": top_name, "achieved": achieved, "peak": peak,
-                "unit": "TFLOP/s", "frac": achieved / peak,
+    top_ms = per_kernel[top_name]["ms_per_launch"]
+    flops_per_launch = top["flops"] / top["launches"]
+    achieved = flops_per_launch / (top_ms / 1e3) / 1e12
+    roofline = {"bound": "tensor", "kernel": top_name, "achieved": achieved, "peak": tensor_peak,
+                "unit": "TFLOP/s", "frac": achieved / tensor_peak,
                 "traffic": traffic_for(top_name, cfg.name),
-                "peak_source": f"{peaks_src} bf16 sustained (kernel timed inside a long step loop)",
-                "launches": top["launches"], "ms_per_launch": per_launch_ms,
+                "peak_source": peak_source,
+                "flops_per_launch": flops_per_launch,
+                "launches_per_step": top["launches"] / kernel_pass_steps,
+                "ms_per_launch": top_ms,
+                "event_ms_per_launch": top["ms"] / top["launches"],
                 "share_of_step": top["ms"] / sum(k["ms"] for k in kinds.values()),
-                "kernel_timing": f"CUDA event pair around every launch on its stream, over "
-                                 f"{kernel_pass_steps} eager steps right after the timed steps "
-                                 "(events between kernels would stop their launch overlap)"}
-    per_kernel = {k: {"launches": v["launches"], "ms_per_launch": v["ms"] / v["launches"],
-                      "tflops": (v["flops"] / v["ms"] / 1e9) if v["flops"] else None,
-                      "gbs": v["bytes"] / v["ms"] / 1e6}
-                  for k, v in kinds.items()}
+                "step_frac": agg["value"] / world / tensor_peak,
+                "kernel_timing": f"in-step time = event-pair time x (step time {step_ms:.4f} ms / "
+                                 f"event times of one step {event_step_ms:.4f} ms); event pairs around "
+                                 f"every launch on its stream over {kernel_pass_steps} eager steps right "
+                                 "after the timed steps (events between kernels stop their launch "
+                                 "overlap, so they are not recorded inside the timed steps)"}
 
     if args.block != "mlp":
         e2e = None
@@ -428,7 +477,7 @@ def bench_ours(args, cfg, world, rank, local):
                           binding, torch)
 
     line = _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, launches,
-                 clocks, working_set, flops_per_step, T, h, F, p)
+                 clocks, working_set, flops_per_step, T, h, F, p, seconds)
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.block == "mlp":
         line["cpu_baseline"] = cpu_baseline(inp, cfg, args.cpu_seconds)
     elif rank == 0:
@@ -512,7 +561,7 @@ def e2e_measure(args, cfg, inp, d, H, Y, Z, gout, ws, p, T, h, dt, dev, stream, 
 
 
 def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, launches, clocks,
-          working_set, flops_per_step, T, h, F, p):
+          working_set, flops_per_step, T, h, F, p, seconds):
     workload = f"{cfg.name}-class TP-MLP fwd+bwd"
     if args.block == "attn-proj":
         workload = f"{cfg.name}-class attention projections (QKV columns + output rows) fwd+bwd"
@@ -534,12 +583,14 @@ def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, la
                    "flops_per_step": flops_per_step, "parallelism": f"replicas x{world}",
                    "cuda_graph": bool(args.graph), "activation": args.activation,
                    "launch_overlap": args.launch_overlap == "on",
+                   "split_policy": args.split_policy,
                    "l2": f"working set {working_set / 2**30:.2f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB "
                          "(inputs larger than L2; no flush)"},
         "frac_of_peak": {"measured_burst": agg["value"] / world / peaks["bf16_tflops"],
-                         "measured_sustained": agg["value"] / world / peaks["bf16_tflops_sustained"],
+                         "measured_sustained": (agg["value"] / world / peaks["bf16_tflops_sustained"]
+                                                if "bf16_tflops_sustained" in peaks else None),
                          "datasheet_dense": agg["value"] / world / DATASHEET_BF16_DENSE_TFLOPS,
-                         "peaks": peaks_src},
+                         "peaks": peaks_src, "timed_region_s": seconds},
         "roofline": roofline,
         "kernels": per_kernel,
         "e2e": e2e,

@@ -32,6 +32,14 @@ def test_bench_json_line_contract():
     for k in ("bound", "achieved", "peak", "unit", "frac", "traffic"):
         assert k in r, k
     assert r["frac"] == pytest.approx(r["achieved"] / r["peak"], rel=1e-6)
+    # the dominant kernel's rate is its algorithmic flops over its in-step time
+    assert r["achieved"] == pytest.approx(r["flops_per_launch"] / (r["ms_per_launch"] / 1e3) / 1e12,
+                                          rel=1e-6)
+    # in-step kernel times add up to the step
+    total = sum(k["ms_per_launch"] * k["launches_per_step"] for k in d["kernels"].values())
+    assert total == pytest.approx(d["ms_per_step"], rel=1e-3)
+    # a 10-step region is far below a second: the burst peak applies
+    assert "burst" in r["peak_source"]
     c = d["cpu_baseline"]
     assert c["kind"] == "oracle" and c["cores"] >= 1 and c["value"] > 0 and c["sample"]
     e = d["e2e"]
