@@ -64,9 +64,12 @@ typedef enum tpmlp_activation { TPMLP_GELU_ERF = 0, TPMLP_GELU_TANH = 1 } tpmlp_
 
 /* Bytes of device workspace that tp_mlp_fwd and tp_mlp_bwd need for these
  * sizes under the current split policy (the larger of the two calls' needs).
- * Returns 0 for invalid sizes. Holds the fp32 shard partials of the two
- * row-parallel products when they are split by shard, and the partial column
- * sums of the bias gradients. */
+ * Returns 0 for invalid sizes. Holds, each part rounded up to 256 bytes:
+ * the fp32 partial tiles and the arrival counters of products whose output
+ * tiles are split over several work units (see tpmlp_set_split_policy;
+ * none when no product splits), and the partial column sums of the bias
+ * gradients. The contents need no initialisation: a call that splits tiles
+ * first zeroes the counters itself. */
 size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt);
 
 /* Forward (column-parallel, then row-parallel):
@@ -177,17 +180,27 @@ const char* tpmlp_strerror(tpmlp_status s);
  * the synchronization itself failed, else TPMLP_OK. */
 tpmlp_status tpmlp_last_device_status(void* stream);
 
-/* How the two row-parallel products (Z = Σ Y_i·B_i and dX = Σ dH_i·A_iᵀ)
- * are scheduled on the tensor-core path:
- *   0 = automatic (split by shard only when the output tiles alone cannot
- *       fill the GPU),
- *   1 = never split: each output tile loops over all shards in ascending
- *       order, accumulating in tensor memory,
- *   2 = always split by shard when F/p is a multiple of 64: each shard's
- *       partial is written in fp32 and the partials are summed in ascending
- *       shard order, then the bias is added.
- * Both orders are deterministic; results agree within rounding. Returns
- * TPMLP_ERR_INVALID for other values. The workspace size depends on it. */
+/* How the tensor-core products are cut into work units. By default every
+ * output tile is one unit whose K loop runs through all k-blocks (for the
+ * two row-parallel products, Z = Σ Y_i·B_i and dX = Σ dH_i·A_iᵀ, through
+ * the shards in ascending order), accumulating in tensor memory. A tile may
+ * instead be split over several units, each covering a consecutive k range;
+ * each writes an fp32 partial, and the last of them to finish adds all the
+ * tile's partials in ascending k order inside the same kernel, then applies
+ * the epilogue (bias, activation, rounding). No unit waits for another.
+ *   0 = automatic: whole tiles in full waves of the GPU's CTA pairs, and
+ *       the remaining tiles' k-blocks cut into one equal segment per pair (a
+ *       stream-K tail) wherever a time model says that is faster,
+ *   1 = whole tiles only,
+ *   2 = the two row-parallel products as one unit per shard and tile when
+ *       F/p is a multiple of 64 (the shards' partials summed in ascending
+ *       shard order, the literal form of the pages' all-reduce); the other
+ *       products as whole tiles,
+ *   3 = the stream-K tail wherever it is valid (for tests and measurement).
+ * Every schedule is deterministic: the same inputs, sizes, policy and GPU
+ * model give bit-identical results. Different schedules agree within
+ * rounding. Returns TPMLP_ERR_INVALID for other values. The workspace size
+ * depends on it. */
 tpmlp_status tpmlp_set_split_policy(int policy);
 int tpmlp_get_split_policy(void);
 
@@ -262,8 +275,14 @@ void tpmlp_profile_reset(void);
  * allocator, or a runtime with a fixed memory budget that forbids
  * allocation after start-up (cudaMalloc and cudaFree can also synchronize
  * the device, which such callers must avoid).
- * Computes exactly what tp_mlp_bwd computes, with the same arguments minus
- * the workspace, and the same requirements. Its only scratch, the partial
+ * Computes the same gradients as tp_mlp_bwd, with the same arguments minus
+ * the workspace, and the same requirements. The results agree within the
+ * library's stated tolerance but not always bit for bit, because the order
+ * of two accumulations can differ: da is summed from per-128-row column-sum
+ * chunks here (tp_mlp_bwd sums two 64-row partials per tile that its GeLU′
+ * epilogue writes when h ≥ 3072), and dX always runs each output tile's K
+ * loop through all shards in tensor memory (tp_mlp_bwd may split that loop
+ * and add the pieces' fp32 partials in ascending order). Its only scratch, the partial
  * column sums of db and da, is a fixed 8 MiB array inside this library
  * (tpmlp_noalloc_scratch_bytes()), held on every GPU that loads the library
  * until the process exits; dX always uses the unsplit schedule (each output
@@ -273,7 +292,10 @@ void tpmlp_profile_reset(void);
  * before any launch. It calls no allocating routine.
  * The first call on each device looks up the array's device address
  * (cudaGetSymbolAddress) with that device current; make that first call
- * before any stream capture. Every call shares the one array: calls whose
+ * before any stream capture. The address is kept for the life of the
+ * process: after cudaDeviceReset on a device, the cached address belongs to
+ * the destroyed context, so do not call this entry point on that device
+ * again in the same process. Every call shares the one array: calls whose
  * kernels overlap on the GPU (on different streams or host threads) race on
  * it and give undefined gradients. Nothing in the array needs to start at
  * zero; each call writes every partial before reading it. */
@@ -284,6 +306,32 @@ tpmlp_status tp_mlp_bwd_noalloc(const void* dZ, const void* X, const void* A, co
 
 /* Size in bytes of the fixed scratch array tp_mlp_bwd_noalloc uses. */
 size_t tpmlp_noalloc_scratch_bytes(void);
+
+/* Diagnostic, host only (launches nothing): the work units the tensor-core
+ * GEMM kernels run for an output of m_blocks × n_blocks tiles and k_blocks
+ * 64-deep k-blocks on `workers` CTA pairs (or single CTAs), under schedule
+ * `sched`: 0 whole tiles; 1 every tile cut into `groups` equal consecutive
+ * k ranges (one per shard group of a row-parallel product); 2 whole tiles
+ * in full waves, then the remaining tiles' k-blocks cut into one equal
+ * segment per worker (a stream-K tail). Writes up to max_units records of
+ * 10 int64 to `out`, in each worker's order: worker, its unit index, m
+ * block, n block, first k-block, end k-block, units sharing the tile,
+ * this unit's place among them (ascending k), the tile's counter index and
+ * this unit's partial-tile slot (both -1 for a whole tile). Returns the
+ * total number of units (which may exceed max_units), or -1 for arguments
+ * the kernels would not run with (a stream-K tail needs tiles not a
+ * multiple of workers and at least 4 k-blocks per segment; shard groups
+ * need k_blocks divisible by groups). */
+int64_t tpmlp_schedule_units(int sched, int m_blocks, int n_blocks, int k_blocks, int groups,
+                             int workers, int64_t* out, int64_t max_units);
+
+/* Diagnostic, host only: the schedule (0 whole tiles, 1 shard groups,
+ * 2 stream-K tail; as tpmlp_schedule_units) that tp_mlp_fwd / tp_mlp_bwd
+ * plan for each of the block's six products, in the order F1 (X·A),
+ * F2 (Σ Y_i·B_i), B2 (dZ·Bᵀ), B3 (Yᵀ·dZ), B4 (Xᵀ·dH), B5 (Σ dH_i·A_iᵀ),
+ * under the current split policy, on the current device (148 SMs when no
+ * device is present). Writes 6 ints to `kinds`. */
+tpmlp_status tpmlp_plan_schedules(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, int* kinds);
 
 /* Library version, major·10000 + minor·100 + patch. */
 int tpmlp_version(void);

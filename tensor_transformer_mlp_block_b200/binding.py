@@ -29,7 +29,7 @@ EXPORTS = (
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
     "tpmlp_profile_read", "tpmlp_profile_reset", "tp_mlp_bwd_noalloc",
-    "tpmlp_noalloc_scratch_bytes", "tpmlp_version",
+    "tpmlp_noalloc_scratch_bytes", "tpmlp_schedule_units", "tpmlp_plan_schedules", "tpmlp_version",
 )
 
 _lib = None
@@ -55,6 +55,11 @@ def lib() -> ctypes.CDLL:
             vp, i64, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_size_t
             L.tpmlp_workspace_size.argtypes = [i64, i64, i64, ctypes.c_int, ctypes.c_int]
             L.tpmlp_workspace_size.restype = sz
+            ci = ctypes.c_int
+            L.tpmlp_schedule_units.argtypes = [ci, ci, ci, ci, ci, ci, ctypes.POINTER(i64), i64]
+            L.tpmlp_schedule_units.restype = i64
+            L.tpmlp_plan_schedules.argtypes = [i64, i64, i64, ci, ci, ctypes.POINTER(ci)]
+            L.tpmlp_plan_schedules.restype = ci
             L.tp_mlp_fwd.argtypes = [vp] * 8 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
             L.tp_mlp_fwd.restype = ctypes.c_int
             L.tp_mlp_bwd.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
@@ -428,3 +433,32 @@ def recompute_activation(H, *, out=None, activation: str = "gelu", stream=None):
                                                  _stream_ptr(H.device, stream)),
                "tp_mlp_recompute_activation")
     return Y
+
+
+# Work-unit schedules of the tensor-core products (tpmlp_schedule_units).
+SCHED_TILES, SCHED_GROUPS, SCHED_STREAMK = 0, 1, 2
+SCHEDULE_FIELDS = ("worker", "local", "mb", "nb", "kb0", "kb1", "pieces", "piece", "key", "slot")
+
+
+def schedule_units(sched: int, m_blocks: int, n_blocks: int, k_blocks: int, workers: int,
+                   groups: int = 1):
+    """The units the GEMM kernels run for this tile grid (host only), as a
+    list of dicts with SCHEDULE_FIELDS; None if the kernels would not run
+    this schedule."""
+    L = lib()
+    n = int(L.tpmlp_schedule_units(sched, m_blocks, n_blocks, k_blocks, groups, workers, None, 0))
+    if n < 0:
+        return None
+    buf = (ctypes.c_int64 * (10 * max(n, 1)))()
+    got = int(L.tpmlp_schedule_units(sched, m_blocks, n_blocks, k_blocks, groups, workers, buf, n))
+    assert got == n
+    return [dict(zip(SCHEDULE_FIELDS, buf[10 * i:10 * i + 10])) for i in range(n)]
+
+
+def plan_schedules(T: int, h: int, F: int, p: int, dtype: torch.dtype = torch.bfloat16):
+    """The schedule planned for F1, F2, B2, B3, B4, B5 at these sizes under
+    the current split policy (host only)."""
+    kinds = (ctypes.c_int * 6)()
+    code = BF16 if dtype == torch.bfloat16 else FP32
+    _check(lib().tpmlp_plan_schedules(T, h, F, p, code, kinds), "tpmlp_plan_schedules")
+    return dict(zip(("F1", "F2", "B2", "B3", "B4", "B5"), list(kinds)))

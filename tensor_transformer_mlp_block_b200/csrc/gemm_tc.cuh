@@ -9,14 +9,25 @@
 // tensor cores read both orientations directly from 128-byte-swizzled shared
 // memory, so no transposed copy is ever made.
 //
-// CTA organisation (192 threads, one CTA per SM, persistent over tiles):
+// CTA organisation (320 threads, one CTA per SM, persistent over tiles):
 //   warp 0      TMA producer: fills a STAGES-deep ring of (A, B) k-blocks
 //   warp 1      tensor-memory allocator and MMA issuer (one thread)
-//   warps 2..5  epilogue: tensor memory -> registers -> fused math -> global
+//   warps 2..9  epilogue: tensor memory -> registers -> fused math -> global
 // The accumulator is double-buffered in tensor memory (2 × BN fp32 columns
 // of 128 lanes), so the epilogue of one tile overlaps the next tile's
-// main loop. Work units are (output tile, K split) pairs handed out
-// round-robin: unit u goes to CTA u mod gridDim.x.
+// main loop. Work units follow one of three schedules (next_unit), which
+// every role of a CTA walks in the same order:
+//   whole tiles    unit u = tile u, handed out round-robin over the CTAs;
+//   shard groups   every tile's K range cut into `groups` equal consecutive
+//                  parts (the row-parallel products' shard groups);
+//   stream-K tail  whole tiles in full waves, then the k-blocks of the
+//                  remaining tiles cut into one equal segment per CTA (pair),
+//                  so that the last wave has no idle SMs.
+// A unit that covers only part of a tile's K range writes its fp32 partial
+// to the workspace and arrives on the tile's counters; the last unit to
+// arrive adds all partials of the tile in ascending k order and runs the
+// epilogue. No unit waits for another, so the sum is the same whichever
+// unit finishes last, and no CTA depends on another CTA being resident.
 //
 // Every wait is bounded (mbar_wait_bounded); a wait that runs out records
 // a timeout in the device status word and the CTA winds down: the producer
@@ -32,7 +43,7 @@ enum EpiKind : int {
     EPI_GELU = 0,        // out0 = H = acc + bias (bf16), out1 = Y = GeLU(H) (bf16)
     EPI_BIAS = 1,        // out0 = acc + bias (element type); bias may be null
     EPI_DGELU = 2,       // out0 = dH = acc · GeLU′(aux) (bf16), aux = saved H (bf16)
-    EPI_F32 = 3,         // out0 (fp32) + split · split_stride = acc
+    EPI_F32 = 3,         // out0 = acc (fp32)
     EPI_GELU_TANH = 4,   // as EPI_GELU with the tanh approximation of GeLU
     EPI_DGELU_TANH = 5,  // as EPI_DGELU with the tanh approximation's derivative
 };
@@ -47,16 +58,23 @@ struct EpiTraits {
     static constexpr bool kBias = (EPI == EPI_BIAS) || kAct;
 };
 
+// Work-unit schedules (see next_unit).
+enum SchedKind : int {
+    SCHED_TILES = 0,    // one unit per output tile
+    SCHED_GROUPS = 1,   // every tile in `groups` consecutive k ranges
+    SCHED_STREAMK = 2,  // whole tiles in full waves, then a stream-K tail
+};
+
 struct GemmArgs {
     int M, N, K;
     int num_m_blocks, num_n_blocks;
-    int splits;        // K splits; work units = tiles × splits
-    int kb_per_split;  // k-blocks of BK per split
     int k_blocks;      // ceil(K / BK)
+    int sched;         // SchedKind
+    int groups;        // SCHED_GROUPS: k ranges per tile
+    int kb_per_group;  // SCHED_GROUPS: k-blocks per range
     void* out0;
     void* out1;
     int64_t ld_out;        // row stride (elements) of out0, out1 and aux
-    int64_t split_stride;  // elements between per-split planes of out0 (EPI_F32)
     const __nv_bfloat16* bias;
     const __nv_bfloat16* aux;
     uint64_t wait_limit_ns;
@@ -64,6 +82,11 @@ struct GemmArgs {
     // output go to colsum_out[r·N + col] (fp32), one row r per 64 rows a
     // computing warp handles in a 128-row CTA tile (see epilogue_role)
     float* colsum_out;
+    // Tiles split over several units (SCHED_GROUPS, the stream-K tail):
+    // fp32 partial tiles (partial_chunk) and 16 arrival counters per split
+    // tile (one per CTA of the pair and epilogue warp), all zero at launch.
+    float* partials;
+    int* counters;
 };
 
 constexpr int kBM = 128;
@@ -89,11 +112,13 @@ struct TileCfg {
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
-__device__ __forceinline__ void unit_coords(const GemmArgs& g, int u, int& mb, int& nb,
-                                            int& split) {
-    const int tiles = g.num_m_blocks * g.num_n_blocks;
-    split = u / tiles;
-    const int t = u - split * tiles;
+// The work schedule below is plain integer arithmetic, compiled for the host
+// too so that the library can list the units it would run (a diagnostic).
+#define TPMLP_HD __host__ __device__ __forceinline__
+
+// Output tile t in grouped raster order: kGroupM m-blocks per group,
+// m fastest inside a group, so that neighbouring units share Bop panels.
+TPMLP_HD void tile_coords(const GemmArgs& g, int t, int& mb, int& nb) {
     const int per_group = kGroupM * g.num_n_blocks;
     const int group = t / per_group;
     const int first_m = group * kGroupM;
@@ -102,6 +127,188 @@ __device__ __forceinline__ void unit_coords(const GemmArgs& g, int u, int& mb, i
     const int idx = t - group * per_group;
     mb = first_m + idx % gm;
     nb = idx / gm;
+}
+
+struct WorkUnit {
+    int mb, nb;    // output tile
+    int kb0, kb1;  // k-blocks [kb0, kb1) of this unit
+    int pieces;    // units sharing the tile (1: the whole K range)
+    int piece;     // this unit's place among them, in ascending k
+    int key;       // split tiles: index of the tile's counters
+    int seg_lo;    // stream-K tail: first segment covering the tile
+};
+
+// Position of one worker (a CTA pair, or a CTA of the one-CTA kernel) in
+// its sequence of units.
+struct WorkIter {
+    int worker, nworkers;
+    int next;       // whole-tile / group units taken so far
+    bool tail;      // in the stream-K segment
+    int64_t cur, end;
+};
+
+TPMLP_HD WorkIter work_iter(int worker, int nworkers) {
+    WorkIter it;
+    it.worker = worker;
+    it.nworkers = nworkers;
+    it.next = 0;
+    it.tail = false;
+    it.cur = it.end = 0;
+    return it;
+}
+
+// Stream-K tail: W k-blocks of the tail tiles (tile-major, k fastest) are cut
+// into P segments; segment j is [begin(j), begin(j + 1)). With W ≥ P no
+// segment is empty. seg_of(x) is the segment that holds k-block x.
+TPMLP_HD int64_t sk_begin(int64_t j, int64_t W, int P) { return j * W / P; }
+TPMLP_HD int sk_seg_of(int64_t x, int64_t W, int P) {
+    return static_cast<int>(((x + 1) * P - 1) / W);
+}
+TPMLP_HD int sk_whole_tiles(const GemmArgs& g, int P) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    return (tiles / P) * P;
+}
+TPMLP_HD int64_t sk_work(const GemmArgs& g, int P) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    return static_cast<int64_t>(tiles - sk_whole_tiles(g, P)) * g.k_blocks;
+}
+
+// The next unit of this worker; false when it has none left.
+TPMLP_HD bool next_unit(const GemmArgs& g, WorkIter& it, WorkUnit& w) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    if (g.sched == SCHED_GROUPS) {
+        const int u = it.worker + it.next * it.nworkers;
+        if (u >= tiles * g.groups) return false;
+        ++it.next;
+        const int s = u / tiles;
+        const int t = u - s * tiles;
+        tile_coords(g, t, w.mb, w.nb);
+        w.kb0 = s * g.kb_per_group;
+        w.kb1 = w.kb0 + g.kb_per_group < g.k_blocks ? w.kb0 + g.kb_per_group : g.k_blocks;
+        w.pieces = g.groups;
+        w.piece = s;
+        w.key = t;
+        w.seg_lo = 0;
+        return true;
+    }
+    const int whole = g.sched == SCHED_STREAMK ? sk_whole_tiles(g, it.nworkers) : tiles;
+    if (!it.tail) {
+        const int u = it.worker + it.next * it.nworkers;
+        if (u < whole) {
+            ++it.next;
+            tile_coords(g, u, w.mb, w.nb);
+            w.kb0 = 0;
+            w.kb1 = g.k_blocks;
+            w.pieces = 1;
+            w.piece = 0;
+            w.key = 0;
+            w.seg_lo = 0;
+            return true;
+        }
+        if (g.sched != SCHED_STREAMK) return false;
+        it.tail = true;
+        const int64_t W = sk_work(g, it.nworkers);
+        it.cur = sk_begin(it.worker, W, it.nworkers);
+        it.end = sk_begin(it.worker + 1, W, it.nworkers);
+    }
+    if (it.cur >= it.end) return false;
+    const int64_t W = sk_work(g, it.nworkers);
+    const int kb = g.k_blocks;
+    const int st = static_cast<int>(it.cur / kb);  // tail tile
+    const int64_t first = static_cast<int64_t>(st) * kb;
+    w.kb0 = static_cast<int>(it.cur - first);
+    const int64_t room = w.kb0 + (it.end - it.cur);
+    w.kb1 = static_cast<int>(room < kb ? room : kb);
+    tile_coords(g, whole + st, w.mb, w.nb);
+    w.seg_lo = sk_seg_of(first, W, it.nworkers);
+    w.pieces = sk_seg_of(first + kb - 1, W, it.nworkers) - w.seg_lo + 1;
+    w.piece = it.worker - w.seg_lo;
+    w.key = st;
+    it.cur += w.kb1 - w.kb0;
+    return true;
+}
+
+// Workspace slot (one partial tile) of piece q of a split tile. Shard groups:
+// one slot per (tile, group). Stream-K tail: two per segment, 2j for the
+// piece that starts where segment j starts, 2j + 1 for the piece that starts
+// at a tile boundary inside it (a segment has at most these two partial
+// pieces; the tiles wholly inside it need no partial).
+TPMLP_HD int64_t partial_slot(const GemmArgs& g, const WorkUnit& w, int q,
+                                                int nworkers) {
+    if (g.sched == SCHED_GROUPS) return static_cast<int64_t>(w.key) * g.groups + q;
+    const int j = w.seg_lo + q;
+    const int64_t begin = sk_begin(j, sk_work(g, nworkers), nworkers);
+    return 2 * static_cast<int64_t>(j) + (begin >= static_cast<int64_t>(w.key) * g.k_blocks ? 0 : 1);
+}
+
+// The 32 × 32 fp32 chunk of a partial tile at tile rows r0.., columns c0..
+// (r0, c0 multiples of 32; a pair tile counts rows over both CTAs): 1024
+// floats in the order the epilogue's registers hold them, float4 j of lane
+// l (row l, columns 4j..4j+3) at index 4·(32·j + l), so that a warp's
+// accesses of one j are 512 contiguous bytes.
+__device__ __forceinline__ float* partial_chunk(const GemmArgs& g, int64_t slot, int tile_rows,
+                                                int bn, int r0, int c0) {
+    return g.partials + slot * static_cast<int64_t>(tile_rows) * bn +
+           static_cast<int64_t>((r0 / 32) * (bn / 32) + c0 / 32) * 1024;
+}
+
+__device__ __forceinline__ void partial_store(float* chunk, const uint32_t (&acc)[32], int lane) {
+    float4* p = reinterpret_cast<float4*>(chunk);
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+        __stcg(p + 32 * j + lane, make_float4(__uint_as_float(acc[4 * j]), __uint_as_float(acc[4 * j + 1]),
+                                              __uint_as_float(acc[4 * j + 2]),
+                                              __uint_as_float(acc[4 * j + 3])));
+}
+
+// acc = Σ_{q = 0 .. pieces-1} partial q, added in ascending q (ascending k).
+__device__ __forceinline__ void partial_sum(const GemmArgs& g, const WorkUnit& w, int nworkers,
+                                            int tile_rows, int bn, int r0, int c0,
+                                            uint32_t (&acc)[32], int lane) {
+    {
+        const float4* p = reinterpret_cast<const float4*>(
+            partial_chunk(g, partial_slot(g, w, 0, nworkers), tile_rows, bn, r0, c0));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = __ldcg(p + 32 * j + lane);
+            acc[4 * j] = __float_as_uint(x.x);
+            acc[4 * j + 1] = __float_as_uint(x.y);
+            acc[4 * j + 2] = __float_as_uint(x.z);
+            acc[4 * j + 3] = __float_as_uint(x.w);
+        }
+    }
+#pragma unroll 1
+    for (int q = 1; q < w.pieces; ++q) {
+        const float4* p = reinterpret_cast<const float4*>(
+            partial_chunk(g, partial_slot(g, w, q, nworkers), tile_rows, bn, r0, c0));
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 x = __ldcg(p + 32 * j + lane);
+            acc[4 * j] = __float_as_uint(__uint_as_float(acc[4 * j]) + x.x);
+            acc[4 * j + 1] = __float_as_uint(__uint_as_float(acc[4 * j + 1]) + x.y);
+            acc[4 * j + 2] = __float_as_uint(__uint_as_float(acc[4 * j + 2]) + x.z);
+            acc[4 * j + 3] = __float_as_uint(__uint_as_float(acc[4 * j + 3]) + x.w);
+        }
+    }
+}
+
+// Arrival of one epilogue warp on its counter of a split tile, after
+// writing its partial chunks. Returns true (in every lane) for the warp of
+// the last unit to arrive, which then reads every partial of the tile; it
+// also puts the counter back to zero for the next launch.
+__device__ __forceinline__ bool partial_arrive(int* ctr, int pieces, int lane) {
+    __threadfence();  // this lane's partial stores are visible device-wide
+    __syncwarp();
+    int old = 0;
+    if (lane == 0) {
+        old = atomicAdd(ctr, 1);
+        __threadfence();  // later loads of the other units' partials see them
+    }
+    old = __shfl_sync(0xffffffffu, old, 0);
+    const bool last = (old == pieces - 1);
+    if (last && lane == 0) atomicExch(ctr, 0);
+    __syncwarp();
+    return last;
 }
 
 // GeLU and its derivative through CUDA's erff/expf (the plain path).
@@ -308,7 +515,7 @@ template <int EPI>
 // and write the column sums to colsum_out row cs_row (if cs_row ≥ 0).
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensorMap* tmO0,
                                                const CUtensorMap* tmO1, const uint32_t (&acc)[32],
-                                               int row0, int col0, int split, uint32_t slot,
+                                               int row0, int col0, uint32_t slot,
                                                int lane, float (&csx)[32], int cs_mode,
                                                int64_t cs_row) {
     const int row = row0 + lane;
@@ -324,7 +531,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0 && any) {
-            tma_store_3d(tmO0, slot, col0, row0, split);
+            tma_store_3d(tmO0, slot, col0, row0, 0);
             bulk_commit();
         }
     } else {
@@ -425,10 +632,10 @@ template <int BN, int EPI, bool PAIR, bool RELAY>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
                                               const CUtensorMap* tmO1, uint32_t tmem_base,
                                               uint64_t* tfull, uint64_t* tempty, uint64_t* xfull,
-                                              uint64_t* xempty, uint8_t* sEpi, int u_first,
-                                              int u_stride, int units, int tile_rows,
-                                              int cta_row_off, volatile int* abort, uint64_t limit,
-                                              int warp, int lane) {
+                                              uint64_t* xempty, uint8_t* sEpi, int worker,
+                                              int nworkers, int tile_rows, int cta_row_off,
+                                              volatile int* abort, uint64_t limit, int warp,
+                                              int lane) {
     constexpr int kChunks = BN / 64;  // 32-column chunks per half of the tile
     const int quad = warp & 3;          // tensor-memory lanes this warp may access
     const int half = (warp - 2) / 4;    // which half of the tile's columns
@@ -443,10 +650,9 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         if (EpiTraits<EPI>::kAct) tma_prefetch_desc(tmO1);
     }
     uint32_t xcount = 0;
-    int local = 0;
-    for (int u = u_first; u < units; u += u_stride, ++local) {
-        int mb, nb, split;
-        unit_coords(g, u, mb, nb, split);
+    WorkIter it = work_iter(worker, nworkers);
+    WorkUnit w;
+    for (int local = 0; next_unit(g, it, w); ++local) {
         const int buf = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         // every lane waits; the warp proceeds only if all lanes saw the
@@ -457,15 +663,26 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
             break;
         }
         tc_fence_after();
-        const int tile_row0 = mb * tile_rows + cta_row_off;
+        const int tile_row0 = w.mb * tile_rows + cta_row_off;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                static_cast<uint32_t>(buf * BN);
+        // a split tile: this unit writes its partial; the last to arrive sums
+        const bool split = w.pieces > 1;
+        const int64_t my_slot = split ? partial_slot(g, w, w.piece, nworkers) : 0;
+        // rows of this warp's own chunks and of the relayed ones, within the tile
+        const int own_r = cta_row_off + quad * 32;
+        const int rel_r = cta_row_off + (quad - 2) * 32;
         bool failed = false;
         float csx[32];  // da partial of the current columns (relay, GeLU′ only)
+        // da partials (relay only): the own rows and the partner's rows of these
+        // columns form one row of colsum_out per computing warp and CTA tile
+        const bool cs_on = RELAY && g.colsum_out != nullptr;
+        const int64_t cs_row =
+            tile_row0 < g.M ? static_cast<int64_t>(tile_row0 / kBM) * 2 + (quad - 2) : -1;
 #pragma unroll 1
         for (int i = 0; i < kChunks; ++i) {
             const int c = half * kChunks + i;
-            const int col0 = nb * BN + c * 32;
+            const int col0 = w.nb * BN + c * 32;
             uint32_t acc[32];
             tmem_ld_32x32b_x32(t_row + c * 32, acc);
             tmem_wait_ld();
@@ -495,13 +712,11 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 ++xcount;
                 continue;
             }
-            // da partials (relay only): the own rows and the partner's rows of these
-            // columns form one row of colsum_out per computing warp and CTA tile
-            const bool cs_on = RELAY && g.colsum_out != nullptr;
-            const int64_t cs_row =
-                tile_row0 < g.M ? static_cast<int64_t>(tile_row0 / kBM) * 2 + (quad - 2) : -1;
-            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, split, slot, lane,
-                                csx, cs_on ? 1 : 0, cs_row);
+            if (split)
+                partial_store(partial_chunk(g, my_slot, tile_rows, BN, own_r, c * 32), acc, lane);
+            else
+                epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane, csx,
+                                    cs_on ? 1 : 0, cs_row);
             if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
                 const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
@@ -520,13 +735,36 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 }
                 mbar_arrive(smem_u32(&xempty[pair_id]));
                 ++xcount;
-                epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, split,
-                                    slot, lane, csx, cs_on ? 2 : 0, cs_row);
+                if (split)
+                    partial_store(partial_chunk(g, my_slot, tile_rows, BN, rel_r, c * 32), pacc, lane);
+                else
+                    epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, slot,
+                                        lane, csx, cs_on ? 2 : 0, cs_row);
             }
         }
         if (failed) {
             raise_timeout(abort);
             break;
+        }
+        if (split && !(RELAY && relay)) {
+            // one counter per split tile, CTA of the pair and epilogue warp
+            int* ctr = g.counters + (static_cast<int64_t>(w.key) * 2 + cta_row_off / kBM) * 8 + (warp - 2);
+            if (partial_arrive(ctr, w.pieces, lane)) {
+#pragma unroll 1
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c = half * kChunks + i;
+                    const int col0 = w.nb * BN + c * 32;
+                    uint32_t acc[32];
+                    partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane);
+                    epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane,
+                                        csx, cs_on ? 1 : 0, cs_row);
+                    if constexpr (RELAY) {
+                        partial_sum(g, w, nworkers, tile_rows, BN, rel_r, c * 32, acc, lane);
+                        epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + (quad - 2) * 32, col0,
+                                            slot, lane, csx, cs_on ? 2 : 0, cs_row);
+                    }
+                }
+            }
         }
     }
     if (lane == 0 && !relay) bulk_wait0();  // this warp's stores are complete before exit
@@ -592,8 +830,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_wait();
     grid_dep_launch();
 
-    const int tiles = g.num_m_blocks * g.num_n_blocks;
-    const int units = tiles * g.splits;
     const uint64_t limit = g.wait_limit_ns;
 
     if (warp == 0) {
@@ -605,12 +841,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t phase = 0;
             int issued = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x) {
-                int mb, nb, split;
-                unit_coords(g, u, mb, nb, split);
-                const int kb0 = split * g.kb_per_split;
-                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
-                for (int kb = kb0; kb < kb1; ++kb) {
+            WorkIter it = work_iter(blockIdx.x, gridDim.x);
+            WorkUnit w;
+            while (ok && next_unit(g, it, w)) {
+                const int mb = w.mb, nb = w.nb;
+                for (int kb = w.kb0; kb < w.kb1; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort, limit)) {
                         raise_timeout(abort);
                         ok = false;
@@ -679,13 +914,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int local = 0;
             bool ok = true;
-            for (int u = blockIdx.x; u < units && ok; u += gridDim.x, ++local) {
-                int mb, nb, split;
-                unit_coords(g, u, mb, nb, split);
-                const int kb0 = split * g.kb_per_split;
-                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
+            WorkIter it = work_iter(blockIdx.x, gridDim.x);
+            WorkUnit w;
+            for (int local = 0; ok && next_unit(g, it, w); ++local) {
+                const int kb0 = w.kb0, kb1 = w.kb1;
                 const int buf = local & 1;
                 const uint32_t aphase = (local >> 1) & 1;
                 if (!mbar_wait_bounded(smem_u32(&tempty[buf]), aphase ^ 1u, abort, limit)) {
@@ -735,7 +968,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue warps
         epilogue_role<BN, EPI, false, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
-                                      blockIdx.x, gridDim.x, units, kBM, 0, abort, limit, warp, lane);
+                                             blockIdx.x, gridDim.x, kBM, 0, abort, limit, warp, lane);
     }
 
     tc_fence_before();

@@ -99,9 +99,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grid_dep_wait();
     grid_dep_launch();
 
-    const int tiles = g.num_m_blocks * g.num_n_blocks;  // num_m_blocks counts 256-row blocks
-    const int units = tiles * g.splits;
-    const uint64_t limit = g.wait_limit_ns;
+    const uint64_t limit = g.wait_limit_ns;  // num_m_blocks counts 256-row blocks
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -114,11 +112,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             const int a_row0 = static_cast<int>(rank) * kBM;
             const int b_col0 = static_cast<int>(rank) * (BN / 2);
-            for (int u = pair; u < units && ok; u += npairs) {
-                int mb, nb, split;
-                unit_coords(g, u, mb, nb, split);
-                const int kb0 = split * g.kb_per_split;
-                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
+            WorkIter it = work_iter(pair, npairs);
+            WorkUnit w;
+            while (ok && next_unit(g, it, w)) {
+                const int mb = w.mb, nb = w.nb;
+                const int kb0 = w.kb0, kb1 = w.kb1;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort, limit)) {
                         raise_timeout(abort);
@@ -188,13 +186,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (leader && lane == 0) {
             int stage = 0;
             uint32_t phase = 0;
-            int local = 0;
             bool ok = true;
-            for (int u = pair; u < units && ok; u += npairs, ++local) {
-                int mb, nb, split;
-                unit_coords(g, u, mb, nb, split);
-                const int kb0 = split * g.kb_per_split;
-                const int kb1 = min(kb0 + g.kb_per_split, g.k_blocks);
+            WorkIter it = work_iter(pair, npairs);
+            WorkUnit w;
+            for (int local = 0; ok && next_unit(g, it, w); ++local) {
+                const int kb0 = w.kb0, kb1 = w.kb1;
                 const int buf = local & 1;
                 const uint32_t aphase = (local >> 1) & 1;
                 if (!mbar_wait_bounded(smem_u32(&tempty[buf]), aphase ^ 1u, abort, limit)) {
@@ -240,8 +236,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
         epilogue_role<BN, EPI, true, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
-                                     pair, npairs, units, kPairM, static_cast<int>(rank) * kBM, abort,
-                                     limit, warp, lane);
+                                            pair, npairs, kPairM, static_cast<int>(rank) * kBM, abort,
+                                            limit, warp, lane);
     }
 
     tc_fence_before();

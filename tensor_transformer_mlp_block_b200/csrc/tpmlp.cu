@@ -6,10 +6,11 @@
 //                        the shard boundary's meaning: every column of H is
 //                        independent, so shards are just column ranges
 //   F2  row-parallel     Z = Σ_i Y_i·B_i + b       the K loop runs over the
-//                        shards in ascending order (in tensor memory), or,
-//                        when the output tiles cannot fill the GPU, each
-//                        shard group writes an fp32 partial and the partials
-//                        are added in ascending order before the bias
+//                        shards in ascending order (in tensor memory); where
+//                        a tile's K range is split over several work units
+//                        (a stream-K tail, or one unit per shard group),
+//                        their fp32 partials are added in ascending order
+//                        inside the same kernel, before the bias
 // and the backward four GEMMs plus two column sums (chain rule):
 //   B2  dH = (dZ·Bᵀ) ⊙ GeLU′(H)   B3  dB = Yᵀ·dZ   B4  dA = Xᵀ·dH
 //   B5  dX = Σ_i dH_i·A_iᵀ (ordered shard sum, as F2)   db, da column sums
@@ -105,17 +106,16 @@ bool make_map(CUtensorMap* m, const void* ptr, int64_t rows, int64_t cols, int b
               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Output of the epilogue's bulk stores: `planes` row-major M × N matrices
-// (one per K split) of bf16 or fp32, written in 32 × 32 boxes; bf16 boxes
-// are 64-byte rows with the 64-byte swizzle, fp32 boxes 128-byte rows with
-// the 128-byte swizzle (the layouts the epilogue stages in shared memory).
-// Box elements outside M × N are not written.
-bool make_out_map(CUtensorMap* m, void* ptr, int64_t planes, int64_t rows, int64_t cols, bool f32) {
+// Output of the epilogue's bulk stores: a row-major M × N matrix of bf16 or
+// fp32, written in 32 × 32 boxes; bf16 boxes are 64-byte rows with the
+// 64-byte swizzle, fp32 boxes 128-byte rows with the 128-byte swizzle (the
+// layouts the epilogue stages in shared memory). Box elements outside
+// M × N are not written. (The map is 3-D with one plane.)
+bool make_out_map(CUtensorMap* m, void* ptr, int64_t rows, int64_t cols, bool f32) {
     EncodeTiledFn fn = encode_fn();
     if (fn == nullptr) return false;
     const cuuint64_t esize = f32 ? 4 : 2;
-    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows),
-                          static_cast<cuuint64_t>(planes)};
+    cuuint64_t dims[3] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows), 1};
     cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * esize,
                              static_cast<cuuint64_t>(rows) * static_cast<cuuint64_t>(cols) * esize};
     cuuint32_t box[3] = {32u, 32u, 1u};
@@ -127,10 +127,10 @@ bool make_out_map(CUtensorMap* m, void* ptr, int64_t planes, int64_t rows, int64
 }
 
 template <int EPI>
-bool make_out_maps(CUtensorMap* o0, CUtensorMap* o1, const GemmArgs& g, int M, int N, int splits) {
+bool make_out_maps(CUtensorMap* o0, CUtensorMap* o1, const GemmArgs& g, int M, int N) {
     const bool f32 = (EPI == EPI_F32);
-    if (!make_out_map(o0, g.out0, f32 ? splits : 1, M, N, f32)) return false;
-    if (EpiTraits<EPI>::kAct) return make_out_map(o1, g.out1, 1, M, N, false);
+    if (!make_out_map(o0, g.out0, M, N, f32)) return false;
+    if (EpiTraits<EPI>::kAct) return make_out_map(o1, g.out1, M, N, false);
     *o1 = *o0;
     return true;
 }
@@ -172,15 +172,15 @@ tpmlp_status launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 // ------------------------------------------------------- per-kernel timing
 
 enum Kind : int {
-    K_F1 = 0, K_F2, K_F2_RED, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_B5_RED, K_MISC,
-    K_L_FWD, K_L_FWD_RED, K_L_DB, K_L_DW, K_L_DX, K_L_DX_RED, K_RECOMP, K_COUNT
+    K_F1 = 0, K_F2, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_MISC,
+    K_L_FWD, K_L_DB, K_L_DW, K_L_DX, K_RECOMP, K_CTR, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
-    "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "F2.split_reduce", "B1.db_colsum",
+    "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "B1.db_colsum",
     "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
-    "B5.dgrad_dX_shard_sum", "B5.split_reduce",       "misc",
-    "L.fwd_gemm_bias",       "L.fwd_split_reduce",    "L.dbias_colsum",  "L.wgrad_dW",
-    "L.dgrad_dX",            "L.dgrad_split_reduce",  "R.recompute_activation",
+    "B5.dgrad_dX_shard_sum", "misc",
+    "L.fwd_gemm_bias",       "L.dbias_colsum",        "L.wgrad_dW",      "L.dgrad_dX",
+    "R.recompute_activation", "S.counter_reset",
 };
 
 struct KindTotals {
@@ -245,12 +245,64 @@ constexpr int kernel_id() {
     return (EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2 + (RELAY ? 1 : 0);
 }
 
+// How a GEMM launch cuts its work into units (see next_unit).
+struct SchedReq {
+    int kind = SCHED_TILES;  // SCHED_TILES, SCHED_GROUPS or SCHED_STREAMK
+    int groups = 1;          // SCHED_GROUPS: consecutive k ranges per tile
+    bool force = false;      // SCHED_STREAMK even where the time model says it does not pay
+};
+
+// Shortest stream-K segment allowed, and the tail's extra cost (partial
+// stores, the last unit's reads and sums, the counter reset), both in
+// k-block times of one worker. Measured on CTA pairs: forcing the tail cost
+// 27–36 µs per product where it saves nothing (7B-class shapes, ~0.43 µs per
+// k-block at power-capped clocks), i.e. ~80 k-blocks.
+constexpr int64_t kSkMinSegmentKb = 4;
+constexpr double kSkOverheadKb = 80.0;
+
+// Whether the stream-K tail is valid for `tiles` output tiles of `kb`
+// k-blocks on P workers and (unless forced) faster than whole tiles. In
+// k-block times of one worker: whole tiles take ceil(tiles/P)·kb; the tail
+// takes floor(tiles/P)·kb + ceil(W/P) + overhead, W = (tiles mod P)·kb.
+bool streamk_pays(int64_t tiles, int64_t kb, int64_t P, bool force) {
+    if (P < 1) return false;
+    const int64_t rem = tiles % P;
+    if (rem == 0) return false;
+    const int64_t W = rem * kb;
+    if (W < P * kSkMinSegmentKb) return false;
+    if (force) return true;
+    const double whole = static_cast<double>((tiles + P - 1) / P) * static_cast<double>(kb);
+    const double tail = static_cast<double>(tiles / P) * static_cast<double>(kb) +
+                        static_cast<double>((W + P - 1) / P) + kSkOverheadKb;
+    return tail < 0.985 * whole;
+}
+
+// Fill g's schedule for at most P workers; returns the number of workers
+// to launch. A split schedule needs the partial-tile workspace.
+int resolve_sched(GemmArgs& g, const SchedReq& req, int64_t P) {
+    const int64_t tiles = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks;
+    g.sched = SCHED_TILES;
+    g.groups = 1;
+    g.kb_per_group = g.k_blocks;
+    const bool have_ws = g.partials != nullptr && g.counters != nullptr;
+    if (req.kind == SCHED_GROUPS && have_ws && req.groups > 1 && g.k_blocks % req.groups == 0) {
+        g.sched = SCHED_GROUPS;
+        g.groups = req.groups;
+        g.kb_per_group = g.k_blocks / req.groups;
+        return static_cast<int>(std::min(tiles * req.groups, P));
+    }
+    if (req.kind == SCHED_STREAMK && have_ws && streamk_pays(tiles, g.k_blocks, P, req.force)) {
+        g.sched = SCHED_STREAMK;
+        return static_cast<int>(P);
+    }
+    return static_cast<int>(std::min(tiles, P));
+}
+
 // D[M, N] = Aop·Bop with Aop stored [M][K] (A_MN = false) or [K][M], Bop
-// stored [N][K] (B_MN = false) or [K][N]. `splits` > 1 splits the k-blocks
-// into equal consecutive ranges (EPI_F32 writes one plane per split).
+// stored [N][K] (B_MN = false) or [K][N].
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
-tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int K, int splits,
-                            GemmArgs g, cudaStream_t st) {
+tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int K,
+                            const SchedReq& req, GemmArgs g, cudaStream_t st) {
     using Cfg = TileCfg<BN>;
     const DeviceInfo* dev = device_info();
     if (dev == nullptr) return TPMLP_ERR_CUDA;
@@ -258,15 +310,13 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
     const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN);
     CUtensorMap tmO0, tmO1;
-    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N, splits)) return TPMLP_ERR_CUDA;
+    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N)) return TPMLP_ERR_CUDA;
     g.M = M;
     g.N = N;
     g.K = K;
     g.num_m_blocks = (M + kBM - 1) / kBM;
     g.num_n_blocks = (N + BN - 1) / BN;
     g.k_blocks = (K + kBK - 1) / kBK;
-    g.splits = splits;
-    g.kb_per_split = (g.k_blocks + splits - 1) / splits;
     g.wait_limit_ns = g_wait_limit_ns.load();
     auto kern = gemm_tc_kernel<BN, A_MN, B_MN, EPI, RELAY>;
     constexpr int id = kernel_id<BN, A_MN, B_MN, EPI, RELAY>();
@@ -282,15 +332,14 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
             g_dev[devn].attr_set |= uint64_t(1) << id;
         }
     }
-    const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
-    const int grid = static_cast<int>(units < dev->num_sms ? units : dev->num_sms);
+    const int grid = resolve_sched(g, req, dev->num_sms);
     return launch_dep(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1, g);
 }
 
 // Same product on CTA pairs: 256 × BN tiles, grid = 2 × (co-resident pairs).
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
-tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int K, int splits,
-                             GemmArgs g, cudaStream_t st) {
+tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int K,
+                             const SchedReq& req, GemmArgs g, cudaStream_t st) {
     using Cfg = Tile2Cfg<BN>;
     const DeviceInfo* dev = device_info();
     if (dev == nullptr) return TPMLP_ERR_CUDA;
@@ -298,15 +347,13 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     const bool okA = A_MN ? make_map(&tmA, Aop, K, M, 64) : make_map(&tmA, Aop, M, K, kBM);
     const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN / 2);
     CUtensorMap tmO0, tmO1;
-    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N, splits)) return TPMLP_ERR_CUDA;
+    if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N)) return TPMLP_ERR_CUDA;
     g.M = M;
     g.N = N;
     g.K = K;
     g.num_m_blocks = (M + kPairM - 1) / kPairM;
     g.num_n_blocks = (N + BN - 1) / BN;
     g.k_blocks = (K + kBK - 1) / kBK;
-    g.splits = splits;
-    g.kb_per_split = (g.k_blocks + splits - 1) / splits;
     g.wait_limit_ns = g_wait_limit_ns.load();
     auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, RELAY>;
     constexpr int id = kernel_id<BN, A_MN, B_MN, EPI, RELAY>();
@@ -339,8 +386,8 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
         }
         max_pairs = d.max_pairs[id];
     }
-    const int64_t units = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks * splits;
-    const int pairs = static_cast<int>(units < max_pairs ? units : max_pairs);
+    // never more workers than the plan sized the workspace for (num_sms / 2)
+    const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2));
     return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
                       g);
 }
@@ -349,12 +396,12 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
 // outputs written once, plus the epilogue's extra input (saved H) and the
 // second output (Y) where the epilogue has them.
 template <int EPI>
-double gemm_bytes(double M, double N, double K, int splits) {
+double gemm_bytes(double M, double N, double K) {
     double b = 2.0 * (M * K + K * N);
     if (EpiTraits<EPI>::kAct) b += 2.0 * 2.0 * M * N;
     if (EPI == EPI_BIAS) b += 2.0 * M * N;
     if (EpiTraits<EPI>::kDAct) b += 2.0 * 2.0 * M * N;
-    if (EPI == EPI_F32) b += 4.0 * M * N * splits;
+    if (EPI == EPI_F32) b += 4.0 * M * N;
     return b;
 }
 
@@ -365,11 +412,11 @@ double gemm_bytes(double M, double N, double K, int splits) {
 // K = 2048; bias store 0.548 -> 0.543 ms at K = 4096, 0.021 -> 0.027 ms at
 // K = 768.
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
-tpmlp_status gemm_tc_pick(const void* Aop, const void* Bop, int M, int N, int K, int splits,
+tpmlp_status gemm_tc_pick(const void* Aop, const void* Bop, int M, int N, int K, const SchedReq& req,
                           const GemmArgs& g, cudaStream_t st) {
     // CTA pairs whenever a 256-row tile is not mostly padding
-    if (M > kBM) return gemm_tc2_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, splits, g, st);
-    return gemm_tc_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, splits, g, st);
+    if (M > kBM) return gemm_tc2_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, req, g, st);
+    return gemm_tc_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, req, g, st);
 }
 
 // Shortest K loop per work unit for which the relaying epilogue pays
@@ -378,15 +425,15 @@ constexpr int kRelayMinKAct = 3072;    // GeLU and GeLU′ epilogues
 constexpr int kRelayMinKPlain = 2048;  // bias and fp32 epilogues
 
 template <int BN, bool A_MN, bool B_MN, int EPI>
-tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K, int splits,
-                     GemmArgs g, cudaStream_t st) {
-    return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K, splits), st, [&] {
-        const int k_per_unit = splits > 1 ? K / splits : K;
+tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K,
+                     const SchedReq& req, GemmArgs g, cudaStream_t st) {
+    return timed(kind, 2.0 * M * N * K, gemm_bytes<EPI>(M, N, K), st, [&] {
+        const int k_per_unit = req.kind == SCHED_GROUPS && req.groups > 1 ? K / req.groups : K;
         const int threshold =
             (EpiTraits<EPI>::kAct || EpiTraits<EPI>::kDAct) ? kRelayMinKAct : kRelayMinKPlain;
         if (k_per_unit < threshold)
-            return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, splits, g, st);
-        return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, splits, g, st);
+            return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, req, g, st);
+        return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, req, g, st);
     });
 }
 
@@ -404,68 +451,103 @@ tpmlp_status gemm_simt(int kind, const SimtArgs& a, cudaStream_t st) {
 
 // ---------------------------------------------------------------- planning
 
-struct Plan {
-    bool tc = false;    // tensor-core path (bf16, h % 8 == 0, F % 8 == 0)
-    int splits = 1;     // shard groups of the two row-parallel products
-    int64_t chunks = 1; // column-sum row chunks
-    size_t off_split = 0, off_cs_h = 0, off_cs_f = 0, total = 0;
-};
-
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
 // Partial rows of da written by the relaying GeLU′ epilogue: two per 128-row
 // CTA tile (one per computing warp, 64 rows each).
 int64_t da_partial_rows(int64_t T) { return T > 0 ? 2 * ((T + kBM - 1) / kBM) : 1; }
 
-// Shard groups S for the two row-parallel products (M = T, N = h, K = F).
-// S = 1 runs each output tile's K loop through all p shards in TMEM; S > 1
-// (a divisor of p, whole k-blocks per shard) gives each group of p/S shards
-// its own work units whose fp32 partials are then summed in order. The
-// automatic policy picks the S with the smallest estimated time:
-//   waves(S) · (k-blocks per unit + per-unit overhead) · t_kblock
-//   + the ordered reduction's bytes (S fp32 planes read, one bf16 written) / HBM rate,
-// with the tile geometry the launcher will use (256-row CTA-pair tiles when
-// T > 128, else 128-row tiles, 256 columns) and one unit per pair / SM in a wave.
-int choose_splits(int64_t T, int64_t h, int64_t F, int p, int num_sms) {
-    const int64_t Fp = F / p;
-    if (p == 1 || Fp % kBK != 0) return 1;
-    const int policy = g_split_policy.load();
-    if (policy == 1) return 1;
-    if (policy == 2) return p;
-    const bool pairs = T > kBM;
-    const int64_t tile_m = pairs ? kPairM : kBM;
-    const int64_t tiles = ((T + tile_m - 1) / tile_m) * ((h + 255) / 256);
-    const int64_t slots = pairs ? num_sms / 2 : num_sms;
-    const double t_kb_us = pairs ? 0.284 : 0.142;  // one 64-deep k-block of a tile
-    const double overhead_kb = 8.0;                 // tile switch, epilogue tail
-    const int64_t k_blocks = (F + kBK - 1) / kBK;
-    int best = 1;
-    double best_us = 0.0;
-    for (int S = 1; S <= p; ++S) {
-        if (p % S != 0) continue;
-        const int64_t units = tiles * S;
-        const int64_t waves = (units + slots - 1) / slots;
-        double us = waves * (static_cast<double>(k_blocks) / S + overhead_kb) * t_kb_us;
-        if (S > 1) us += 3.0 + static_cast<double>(T) * h * (4.0 * S + 2.0) / 5.0e6;
-        if (S == 1 || us < best_us) {
-            best = S;
-            best_us = us;
-        }
+// Workspace a call's split tiles need: fp32 partial tiles and arrival
+// counters (16 per split tile). Shared by the call's products, which run
+// one after another on the stream; every counter is back at zero when a
+// launch completes, and the call zeroes them once before its first launch.
+struct SplitSpace {
+    size_t partial_bytes = 0, counter_bytes = 0;
+    void need(size_t part, size_t ctr) {
+        partial_bytes = std::max(partial_bytes, part);
+        counter_bytes = std::max(counter_bytes, ctr);
     }
-    return best;
+};
+
+// Schedule of one tensor-core product (M × N output, K deep) under the
+// current policy (tpmlp_set_split_policy):
+//   0  stream-K tail where the time model says it pays (streamk_pays);
+//   1  whole tiles only;
+//   2  a row-parallel product (shard_groups > 1: p shards of whole k-blocks)
+//      as one unit per shard and tile, the shards' partials added in
+//      ascending order; other products as whole tiles;
+//   3  stream-K tail wherever it is valid (for tests and measurement).
+// The geometry is the launcher's: CTA pairs with 256-row tiles and
+// num_sms / 2 workers when M > 128, else one CTA per 128-row tile and
+// num_sms workers; 256-column tiles.
+SchedReq plan_sched(int64_t M, int64_t N, int64_t K, int shard_groups, int num_sms, SplitSpace* sp) {
+    SchedReq r;
+    const int policy = g_split_policy.load();
+    const bool pairs = M > kBM;
+    const int64_t tile_rows = pairs ? kPairM : kBM;
+    const int64_t workers = pairs ? num_sms / 2 : num_sms;
+    const int64_t tiles = ((M + tile_rows - 1) / tile_rows) * ((N + 255) / 256);
+    const int64_t kb = (K + kBK - 1) / kBK;
+    const size_t tile_bytes = static_cast<size_t>(tile_rows) * 256 * sizeof(float);
+    if (policy == 2 && shard_groups > 1 && kb % shard_groups == 0) {
+        r.kind = SCHED_GROUPS;
+        r.groups = shard_groups;
+        sp->need(static_cast<size_t>(tiles) * shard_groups * tile_bytes,
+                 static_cast<size_t>(tiles) * 16 * sizeof(int));
+        return r;
+    }
+    if ((policy == 0 || policy == 3) && streamk_pays(tiles, kb, workers, policy == 3)) {
+        r.kind = SCHED_STREAMK;
+        r.force = (policy == 3);
+        sp->need(static_cast<size_t>(2 * workers) * tile_bytes,
+                 static_cast<size_t>(workers) * 16 * sizeof(int));
+    }
+    return r;
 }
+
+// Shard groups of a row-parallel product whose K = p shards of Fp: p when
+// every shard is whole k-blocks, else none (the K loop runs through all shards).
+int shard_groups(int64_t K, int p) {
+    return (p > 1 && K % p == 0 && (K / p) % kBK == 0) ? p : 0;
+}
+
+int plan_num_sms() {
+    if (const DeviceInfo* d = device_info()) return d->num_sms;
+    return 148;
+}
+
+struct Plan {
+    bool tc = false;    // tensor-core path (bf16, h % 8 == 0, F % 8 == 0)
+    SchedReq f1, f2, b2, b3, b4, b5;
+    bool fwd_split = false, bwd_split = false;  // some product of the call splits tiles
+    int64_t chunks = 1; // column-sum row chunks
+    size_t off_part = 0, off_ctr = 0, ctr_bytes = 0, off_cs_h = 0, off_cs_f = 0, total = 0;
+};
 
 bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl) {
     if (T < 0 || h < 1 || F < 1 || p < 1 || F % p != 0) return false;
     if (dt != TPMLP_BF16 && dt != TPMLP_FP32) return false;
     pl->tc = (dt == TPMLP_BF16) && (h % 8 == 0) && (F % 8 == 0);
-    int num_sms = 148;
-    if (const DeviceInfo* d = device_info()) num_sms = d->num_sms;
-    pl->splits = pl->tc ? choose_splits(T, h, F, p, num_sms) : 1;
+    SplitSpace sp;
+    if (pl->tc && T > 0) {
+        const int sms = plan_num_sms();
+        pl->f1 = plan_sched(T, F, h, 0, sms, &sp);                   // X·A
+        pl->f2 = plan_sched(T, h, F, shard_groups(F, p), sms, &sp);  // Σ Y_i·B_i
+        pl->b2 = plan_sched(T, F, h, 0, sms, &sp);                   // dZ·Bᵀ
+        pl->b3 = plan_sched(F, h, T, 0, sms, &sp);                   // Yᵀ·dZ
+        pl->b4 = plan_sched(h, F, T, 0, sms, &sp);                   // Xᵀ·dH
+        pl->b5 = plan_sched(T, h, F, shard_groups(F, p), sms, &sp);  // Σ dH_i·A_iᵀ
+        pl->fwd_split = pl->f1.kind != SCHED_TILES || pl->f2.kind != SCHED_TILES;
+        pl->bwd_split = pl->b2.kind != SCHED_TILES || pl->b3.kind != SCHED_TILES ||
+                        pl->b4.kind != SCHED_TILES || pl->b5.kind != SCHED_TILES;
+    }
     pl->chunks = T > 0 ? (T + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk : 1;
     size_t off = 0;
-    pl->off_split = off;
-    if (pl->splits > 1) off += round256(static_cast<size_t>(pl->splits) * T * h * sizeof(float));
+    pl->off_part = off;
+    off += round256(sp.partial_bytes);
+    pl->off_ctr = off;
+    pl->ctr_bytes = round256(sp.counter_bytes);
+    off += pl->ctr_bytes;
     pl->off_cs_h = off;
     off += round256(static_cast<size_t>(pl->chunks) * h * sizeof(float));
     pl->off_cs_f = off;
@@ -537,22 +619,6 @@ tpmlp_status colsum_finish(int kind, const float* partial, int64_t rows, int64_t
     });
 }
 
-tpmlp_status reduce_splits_launch(const float* ws, int splits, int64_t M, int64_t N,
-                                  const void* bias, void* out, cudaStream_t st) {
-    const int64_t groups = M * (N / 8);
-    const int64_t blocks =
-        clamp_grid((groups + 255) / 256, resident_blocks<reduce_splits_bf16_kernel>(256));
-    return launch_dep(reduce_splits_bf16_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st,
-                      ws, splits, M * N, static_cast<const __nv_bfloat16*>(bias),
-                      static_cast<__nv_bfloat16*>(out), M, N);
-}
-
-tpmlp_status reduce_splits(int kind, const float* ws, int splits, int64_t M, int64_t N,
-                           const void* bias, void* out, cudaStream_t st) {
-    return timed(kind, 0.0, 4.0 * splits * double(M) * N + 2.0 * double(M) * N, st,
-                 [&] { return reduce_splits_launch(ws, splits, M, N, bias, out, st); });
-}
-
 // One launch of recompute_act_kernel over n elements: a thread-iteration
 // takes two 8-element groups (VEC) or one element; no more blocks than the
 // device holds at once.
@@ -565,12 +631,25 @@ tpmlp_status launch_recompute(const void* H, void* Y, int64_t n, cudaStream_t st
                       static_cast<const T*>(H), static_cast<T*>(Y), n);
 }
 
-tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st) {
+tpmlp_status zero_f32(float* p, int64_t n, cudaStream_t st, int kind = K_MISC) {
     if (n <= 0) return TPMLP_OK;
-    return timed(K_MISC, 0.0, 4.0 * n, st, [&] {
+    return timed(kind, 0.0, 4.0 * n, st, [&] {
         const int64_t blocks = clamp_grid((n + 255) / 256, resident_blocks<zero_f32_kernel>(256));
         return launch_dep(zero_f32_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, st, p, n);
     });
+}
+
+// Arrival counters of split tiles: zeroed once at the start of a call whose
+// plan splits tiles (each launch leaves them at zero again).
+tpmlp_status reset_counters(void* workspace, size_t off, size_t bytes, cudaStream_t st) {
+    float* p = reinterpret_cast<float*>(static_cast<char*>(workspace) + off);  // 0.0f is all-zero bits
+    return zero_f32(p, static_cast<int64_t>(bytes / sizeof(float)), st, K_CTR);
+}
+
+// Workspace pointers of a call's split tiles.
+void set_split_space(GemmArgs& g, void* workspace, size_t off_part, size_t off_ctr) {
+    g.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + off_part);
+    g.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + off_ctr);
 }
 
 #define TPMLP_TRY(expr)                         \
@@ -598,13 +677,15 @@ tpmlp_status common_checks(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype d
 
 // Plan of a linear layer Y = X·W + bias (X: T × K, W: K × N), W split into
 // p shards by columns (split 0) or rows (split 1). The product carrying a
-// shard sum (the forward for rows, dX of the backward for columns) may be
-// split by shard like the MLP's row-parallel products.
+// shard sum (the forward for rows, dX of the backward for columns) may run
+// one unit per shard and tile like the MLP's row-parallel products; every
+// product may take a stream-K tail.
 struct LinPlan {
     bool tc = false;
-    int splits_fwd = 1, splits_bwd = 1;
+    SchedReq fwd, dw, dx;
+    bool fwd_split = false, bwd_split = false;
     int64_t chunks = 1;
-    size_t off_split = 0, off_cs = 0, total = 0;
+    size_t off_part = 0, off_ctr = 0, ctr_bytes = 0, off_cs = 0, total = 0;
 };
 
 bool make_lin_plan(int64_t T, int64_t K, int64_t N, int p, int split, tpmlp_dtype dt, LinPlan* pl) {
@@ -613,19 +694,20 @@ bool make_lin_plan(int64_t T, int64_t K, int64_t N, int p, int split, tpmlp_dtyp
     if (split == 1 && K % p != 0) return false;
     if (dt != TPMLP_BF16 && dt != TPMLP_FP32) return false;
     pl->tc = (dt == TPMLP_BF16) && (K % 8 == 0) && (N % 8 == 0);
-    int num_sms = 148;
-    if (const DeviceInfo* d = device_info()) num_sms = d->num_sms;
-    if (pl->tc) {
-        if (split == 1) pl->splits_fwd = choose_splits(T, N, K, p, num_sms);
-        else pl->splits_bwd = choose_splits(T, K, N, p, num_sms);
+    SplitSpace sp;
+    if (pl->tc && T > 0) {
+        const int sms = plan_num_sms();
+        pl->fwd = plan_sched(T, N, K, split == 1 ? shard_groups(K, p) : 0, sms, &sp);
+        pl->dw = plan_sched(K, N, T, 0, sms, &sp);
+        pl->dx = plan_sched(T, K, N, split == 0 ? shard_groups(N, p) : 0, sms, &sp);
+        pl->fwd_split = pl->fwd.kind != SCHED_TILES;
+        pl->bwd_split = pl->dw.kind != SCHED_TILES || pl->dx.kind != SCHED_TILES;
     }
     pl->chunks = T > 0 ? (T + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk : 1;
-    size_t split_bytes = 0;
-    if (pl->splits_fwd > 1) split_bytes = static_cast<size_t>(pl->splits_fwd) * T * N * sizeof(float);
-    if (pl->splits_bwd > 1)
-        split_bytes = std::max(split_bytes, static_cast<size_t>(pl->splits_bwd) * T * K * sizeof(float));
-    pl->off_split = 0;
-    pl->off_cs = round256(split_bytes);
+    pl->off_part = 0;
+    pl->off_ctr = round256(sp.partial_bytes);
+    pl->ctr_bytes = round256(sp.counter_bytes);
+    pl->off_cs = pl->off_ctr + pl->ctr_bytes;
     pl->total = pl->off_cs + round256(static_cast<size_t>(pl->chunks) * N * sizeof(float));
     return true;
 }
@@ -655,20 +737,15 @@ tpmlp_status linear_fwd_impl(const void* X, const void* W, const void* bias, voi
     if (pl.tc) {
         for (const void* q : {X, W, bias, static_cast<const void*>(Y)})
             if (q && !aligned16(q)) return TPMLP_ERR_ALIGN;
-        // Aop = X [T][K] (K-major), Bop = W [K][N] (MN-major)
+        if (pl.fwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
+        // Aop = X [T][K] (K-major), Bop = W [K][N] (MN-major); for the row split
+        // the K loop (or the units' partials) runs through the shards in order
         GemmArgs g{};
-        if (pl.splits_fwd == 1) {
-            g.out0 = Y;
-            g.ld_out = N;
-            g.bias = static_cast<const __nv_bfloat16*>(bias);
-            return gemm_tc<256, false, true, EPI_BIAS>(K_L_FWD, X, W, iT, iN, iK, 1, g, st);
-        }
-        float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
-        g.out0 = ws;
+        set_split_space(g, workspace, pl.off_part, pl.off_ctr);
+        g.out0 = Y;
         g.ld_out = N;
-        g.split_stride = T * N;
-        TPMLP_TRY((gemm_tc<256, false, true, EPI_F32>(K_L_FWD, X, W, iT, iN, iK, pl.splits_fwd, g, st)));
-        return reduce_splits(K_L_FWD_RED, ws, pl.splits_fwd, T, N, bias, Y, st);
+        g.bias = static_cast<const __nv_bfloat16*>(bias);
+        return gemm_tc<256, false, true, EPI_BIAS>(K_L_FWD, X, W, iT, iN, iK, pl.fwd, g, st);
     }
     SimtArgs a{};
     a.M = iT; a.N = iN; a.K = iK;
@@ -697,26 +774,21 @@ tpmlp_status linear_bwd_impl(const void* dY, const void* X, const void* W, void*
         for (const void* q : {dY, X, W, static_cast<const void*>(dX), static_cast<const void*>(dW),
                               static_cast<const void*>(dbias)})
             if (!aligned16(q)) return TPMLP_ERR_ALIGN;
+        if (pl.bwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         TPMLP_TRY(colsum(K_L_DB, static_cast<const __nv_bfloat16*>(dY), T, N, pl.chunks, cs, dbias, st));
         // dW = Xᵀ·dY: Aop = X [T][K] (MN-major, M = K), Bop = dY [T][N] (MN-major)
         GemmArgs gw{};
+        set_split_space(gw, workspace, pl.off_part, pl.off_ctr);
         gw.out0 = dW;
         gw.ld_out = N;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_L_DW, X, dY, iK, iN, iT, 1, gw, st)));
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_L_DW, X, dY, iK, iN, iT, pl.dw, gw, st)));
         // dX = dY·Wᵀ: Aop = dY [T][N] (K-major), Bop = W [K][N] read as [N' = K][K' = N] (K-major);
         // for the column split this is the shard sum over the N dimension
         GemmArgs gx{};
-        if (pl.splits_bwd == 1) {
-            gx.out0 = dX;
-            gx.ld_out = K;
-            return gemm_tc<256, false, false, EPI_BIAS>(K_L_DX, dY, W, iT, iK, iN, 1, gx, st);
-        }
-        float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
-        gx.out0 = ws;
+        set_split_space(gx, workspace, pl.off_part, pl.off_ctr);
+        gx.out0 = dX;
         gx.ld_out = K;
-        gx.split_stride = T * K;
-        TPMLP_TRY((gemm_tc<256, false, false, EPI_F32>(K_L_DX, dY, W, iT, iK, iN, pl.splits_bwd, gx, st)));
-        return reduce_splits(K_L_DX_RED, ws, pl.splits_bwd, T, K, nullptr, dX, st);
+        return gemm_tc<256, false, false, EPI_BIAS>(K_L_DX, dY, W, iT, iK, iN, pl.dx, gx, st);
     }
     // dW = Xᵀ·dY: Aop(k, t) = X[t][k], Bop(t, n) = dY[t][n]
     SimtArgs w{};
@@ -759,29 +831,28 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
                               static_cast<const void*>(Z)})
             if (q && !aligned16(q)) return TPMLP_ERR_ALIGN;
         const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
+        // without F2 (activation recompute) there is no workspace: whole tiles
+        const SchedReq f1 = with_f2 ? pl.f1 : SchedReq{};
+        if (with_f2 && pl.fwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         // F1: H = X·A + a, Y = GeLU(H). Aop = X [T][h] (K-major), Bop = A [h][F] (MN-major).
         GemmArgs g1{};
+        if (with_f2) set_split_space(g1, workspace, pl.off_part, pl.off_ctr);
         g1.out0 = H;
         g1.out1 = Y;
         g1.ld_out = F;
         g1.bias = static_cast<const __nv_bfloat16*>(a);
-        TPMLP_TRY((gemm_tc<256, false, true, EPI_ACT>(K_F1, X, A, iT, iF, ih, 1, g1, st)));
+        TPMLP_TRY((gemm_tc<256, false, true, EPI_ACT>(K_F1, X, A, iT, iF, ih, f1, g1, st)));
         if (!with_f2) return TPMLP_OK;
         // F2: Z = Σ_i Y_i·B_i + b. Aop = Y [T][F] (K-major), Bop = B [F][h] (MN-major).
+        // Each tile's K loop runs through the shards in ascending order; where
+        // the schedule splits a tile, the units' partials are added in ascending
+        // order in the epilogue of the last one, then b once.
         GemmArgs g2{};
-        if (pl.splits == 1) {
-            g2.out0 = Z;
-            g2.ld_out = h;
-            g2.bias = static_cast<const __nv_bfloat16*>(b);
-            TPMLP_TRY((gemm_tc<256, false, true, EPI_BIAS>(K_F2, Y, B, iT, ih, iF, 1, g2, st)));
-        } else {
-            float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
-            g2.out0 = ws;
-            g2.ld_out = h;
-            g2.split_stride = T * h;
-            TPMLP_TRY((gemm_tc<256, false, true, EPI_F32>(K_F2, Y, B, iT, ih, iF, pl.splits, g2, st)));
-            TPMLP_TRY(reduce_splits(K_F2_RED, ws, pl.splits, T, h, b, Z, st));
-        }
+        set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
+        g2.out0 = Z;
+        g2.ld_out = h;
+        g2.bias = static_cast<const __nv_bfloat16*>(b);
+        TPMLP_TRY((gemm_tc<256, false, true, EPI_BIAS>(K_F2, Y, B, iT, ih, iF, pl.f2, g2, st)));
         return TPMLP_OK;
     }
     // plain CUDA-core path: fp32, or bf16 with h or F not a multiple of 8
@@ -834,6 +905,7 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
             if (!aligned16(q)) return TPMLP_ERR_ALIGN;
         const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
         const __nv_bfloat16* dZb = static_cast<const __nv_bfloat16*>(dZ);
+        if (pl.bwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         // db = 1ᵀ·dZ
         TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
@@ -843,11 +915,12 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // the extra epilogue work costs more than the separate pass.
         const bool fused_da = h >= kRelayMinKAct;
         GemmArgs g2{};
+        set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
         g2.colsum_out = fused_da ? cs_f : nullptr;
-        TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, pl.b2, g2, st)));
         // da = 1ᵀ·dH
         if (fused_da)
             TPMLP_TRY(colsum_finish(K_B2_DA, cs_f, da_partial_rows(T), F, da, st));
@@ -856,28 +929,22 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
                              da, st));
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
         GemmArgs g3{};
+        set_split_space(g3, workspace, pl.off_part, pl.off_ctr);
         g3.out0 = dB;
         g3.ld_out = h;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, 1, g3, st)));
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, pl.b3, g3, st)));
         // B4: dA = Xᵀ·dH. Aop = X [T][h] (MN-major, M = h), Bop = dH [T][F] (MN-major).
         GemmArgs g4{};
+        set_split_space(g4, workspace, pl.off_part, pl.off_ctr);
         g4.out0 = dA;
         g4.ld_out = F;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, 1, g4, st)));
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, pl.b4, g4, st)));
         // B5: dX = Σ_i dH_i·A_iᵀ. Aop = dH [T][F] (K-major), Bop = A [h][F] (K-major).
         GemmArgs g5{};
-        if (pl.splits == 1) {
-            g5.out0 = dX;
-            g5.ld_out = h;
-            TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, 1, g5, st)));
-        } else {
-            float* ws = reinterpret_cast<float*>(static_cast<char*>(workspace) + pl.off_split);
-            g5.out0 = ws;
-            g5.ld_out = h;
-            g5.split_stride = T * h;
-            TPMLP_TRY((gemm_tc<256, false, false, EPI_F32>(K_B5, dH, A, iT, ih, iF, pl.splits, g5, st)));
-            TPMLP_TRY(reduce_splits(K_B5_RED, ws, pl.splits, T, h, nullptr, dX, st));
-        }
+        set_split_space(g5, workspace, pl.off_part, pl.off_ctr);
+        g5.out0 = dX;
+        g5.ld_out = h;
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, pl.b5, g5, st)));
         return TPMLP_OK;
     }
     const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
@@ -1073,7 +1140,7 @@ tpmlp_status tpmlp_last_device_status(void* stream) {
 }
 
 tpmlp_status tpmlp_set_split_policy(int policy) {
-    if (policy < 0 || policy > 2) return TPMLP_ERR_INVALID;
+    if (policy < 0 || policy > 3) return TPMLP_ERR_INVALID;
     g_split_policy.store(policy);
     return TPMLP_OK;
 }
@@ -1153,7 +1220,62 @@ void tpmlp_profile_reset(void) {
     for (KindTotals& t : g_prof) t = KindTotals{};
 }
 
-int tpmlp_version(void) { return 100; }
+int64_t tpmlp_schedule_units(int sched, int m_blocks, int n_blocks, int k_blocks, int groups,
+                             int workers, int64_t* out, int64_t max_units) {
+    if (m_blocks < 1 || n_blocks < 1 || k_blocks < 1 || workers < 1 || max_units < 0) return -1;
+    if (max_units > 0 && out == nullptr) return -1;
+    GemmArgs g{};
+    g.num_m_blocks = m_blocks;
+    g.num_n_blocks = n_blocks;
+    g.k_blocks = k_blocks;
+    g.groups = 1;
+    g.kb_per_group = k_blocks;
+    const int64_t tiles = static_cast<int64_t>(m_blocks) * n_blocks;
+    if (tiles > (int64_t(1) << 30)) return -1;
+    if (sched == SCHED_TILES) {
+        g.sched = SCHED_TILES;
+    } else if (sched == SCHED_GROUPS) {
+        if (groups < 2 || k_blocks % groups != 0) return -1;
+        g.sched = SCHED_GROUPS;
+        g.groups = groups;
+        g.kb_per_group = k_blocks / groups;
+    } else if (sched == SCHED_STREAMK) {
+        if (!streamk_pays(tiles, k_blocks, workers, true)) return -1;
+        g.sched = SCHED_STREAMK;
+    } else {
+        return -1;
+    }
+    int64_t n = 0;
+    for (int wk = 0; wk < workers; ++wk) {
+        WorkIter it = work_iter(wk, workers);
+        WorkUnit w;
+        for (int local = 0; next_unit(g, it, w); ++local, ++n) {
+            if (n >= max_units) continue;
+            int64_t* r = out + 10 * n;
+            r[0] = wk;
+            r[1] = local;
+            r[2] = w.mb;
+            r[3] = w.nb;
+            r[4] = w.kb0;
+            r[5] = w.kb1;
+            r[6] = w.pieces;
+            r[7] = w.piece;
+            r[8] = w.pieces > 1 ? w.key : -1;
+            r[9] = w.pieces > 1 ? partial_slot(g, w, w.piece, workers) : -1;
+        }
+    }
+    return n;
+}
+
+tpmlp_status tpmlp_plan_schedules(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, int* kinds) {
+    Plan pl;
+    if (kinds == nullptr || !make_plan(T, h, F, p, dt, &pl)) return TPMLP_ERR_INVALID;
+    const SchedReq* r[6] = {&pl.f1, &pl.f2, &pl.b2, &pl.b3, &pl.b4, &pl.b5};
+    for (int i = 0; i < 6; ++i) kinds[i] = r[i]->kind;
+    return TPMLP_OK;
+}
+
+int tpmlp_version(void) { return 200; }
 
 }  // extern "C"
 
@@ -1241,7 +1363,8 @@ tpmlp_status tp_mlp_bwd_noalloc(const void* dZ, const void* X, const void* A, co
         return TPMLP_OK;
     }
     // Every partial the column sums use is written before it is read, so
-    // nothing in the scratch has to start at zero.
+    // nothing in the scratch has to start at zero. Every product runs as
+    // whole tiles (no partial tiles, no counters).
     float* cs_h = static_cast<float*>(scratch);
     float* cs_f = reinterpret_cast<float*>(static_cast<char*>(scratch) + cs_h_bytes);
     const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
@@ -1251,20 +1374,20 @@ tpmlp_status tp_mlp_bwd_noalloc(const void* dZ, const void* X, const void* A, co
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
-        TPMLP_TRY((gemm_tc<256, false, false, EPI_DGELU>(K_B2, dZ, B, iT, iF, ih, 1, g2, st)));
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_DGELU>(K_B2, dZ, B, iT, iF, ih, SchedReq{}, g2, st)));
         TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f, da, st));
         GemmArgs g3{};
         g3.out0 = dB;
         g3.ld_out = h;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, 1, g3, st)));
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, SchedReq{}, g3, st)));
         GemmArgs g4{};
         g4.out0 = dA;
         g4.ld_out = F;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, 1, g4, st)));
+        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, SchedReq{}, g4, st)));
         GemmArgs g5{};
         g5.out0 = dX;
         g5.ld_out = h;
-        TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, 1, g5, st)));
+        TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, SchedReq{}, g5, st)));
         return TPMLP_OK;
     }
     SimtArgs s2{};

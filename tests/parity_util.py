@@ -80,8 +80,9 @@ def _u(key: str, dtype: str) -> float:
     return UNIT_ROUNDOFF[dtype] if key.split("[")[0] in STORED else 0.0
 
 
-def run_gpu(inp: dict, p: int, device="cuda:0", activation: str = "gelu"):
-    """Forward + backward on the GPU through the binding. Returns CPU tensors."""
+def run_gpu(inp: dict, p: int, device="cuda:0", activation: str = "gelu", keep_on_device=False):
+    """Forward + backward on the GPU through the binding. Returns CPU tensors
+    (or the device tensors with keep_on_device)."""
     from tensor_transformer_mlp_block_b200 import binding
     d = {k: v.to(device) for k, v in inp.items()}
     H, Y, Z = binding.forward(d["X"], d["A"], d["a"], d["B"], d["b"], p, activation=activation)
@@ -90,6 +91,8 @@ def run_gpu(inp: dict, p: int, device="cuda:0", activation: str = "gelu"):
     st = binding.last_device_status(device=device)
     assert st == 0, f"device status {st}"
     out = dict(H=H, Y=Y, Z=Z, **g)
+    if keep_on_device:
+        return out
     return {k: v.cpu() for k, v in out.items()}
 
 
@@ -114,17 +117,21 @@ def compare_full(gpu: dict, ref: dict, dtype: str, keys=None) -> dict:
     return errs
 
 
-def compare_sampled(gpu: dict, inp: dict, R, J, dtype: str, act: int = 0) -> dict:
-    """Compare on token rows R and hidden columns J, each computed exactly by
-    the oracle (rows: H, Y, Z, dH, dX; columns: H, Y, dH, dA, da, dB), plus
-    db in full."""
+def oracle_sampled(inp: dict, R, J, act: int = 0) -> dict:
+    """The oracle's exact values on token rows R (H, Y, Z, dH, dX) and hidden
+    columns J (H, Y, dH, dA, da, dB), plus db in full."""
     n = {k: to_np(v) for k, v in inp.items()}
     R = np.asarray(R)
     J = np.asarray(J)
     r = oracle.rows(n["X"], n["A"], n["a"], n["B"], n["b"], n["dZ"], R, act)
     # the column subset needs only A[:, J], a[J], B[J, :]
     c = oracle.cols(n["X"], n["A"][:, J], n["a"][J], n["B"][J, :], n["dZ"], np.arange(len(J)), act)
-    db = oracle.colsum(n["dZ"])
+    return {"R": R, "J": J, "rows": r, "cols": c, "db": oracle.colsum(n["dZ"])}
+
+
+def compare_to_sampled(gpu: dict, ref: dict, dtype: str) -> dict:
+    """Compare GPU outputs (CPU or CUDA tensors) with oracle_sampled's values."""
+    R, J, r, c = ref["R"], ref["J"], ref["rows"], ref["cols"]
     tol = TOL[dtype]
     errs = {}
     for k in ("H", "Y", "Z", "dH", "dX"):
@@ -134,8 +141,15 @@ def compare_sampled(gpu: dict, inp: dict, R, J, dtype: str, act: int = 0) -> dic
     errs["dA[:,J]"] = rel_err(to_np(gpu["dA"][:, J]), c["dA"])
     errs["da[J]"] = rel_err(to_np(gpu["da"][J]), c["da"])
     errs["dB[J]"] = rel_err(to_np(gpu["dB"][J]), c["dB"])
-    errs["db"] = rel_err(to_np(gpu["db"]), db)
+    errs["db"] = rel_err(to_np(gpu["db"]), ref["db"])
     bad = {k: e for k, e in errs.items() if not e <= tol}
     assert not bad, f"outside {tol}·rms: {bad} (all: {errs})"
     print("parity", {k: round(v, 5) for k, v in errs.items()})
     return errs
+
+
+def compare_sampled(gpu: dict, inp: dict, R, J, dtype: str, act: int = 0) -> dict:
+    """Compare on token rows R and hidden columns J, each computed exactly by
+    the oracle (rows: H, Y, Z, dH, dX; columns: H, Y, dH, dA, da, dB), plus
+    db in full."""
+    return compare_to_sampled(gpu, oracle_sampled(inp, R, J, act), dtype)

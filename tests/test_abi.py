@@ -93,59 +93,81 @@ def test_workspace_size_host_logic(lib):
     binding.set_split_policy(2)
     split = binding.workspace_size(1024, 512, 2048, 4)
     binding.set_split_policy(0)
-    # forcing the shard split adds p fp32 planes of T×h
+    # one unit per shard and tile adds p fp32 partial tiles per output tile
     assert split - base >= 4 * 1024 * 512 * 4
     assert base % 256 == 0 and split % 256 == 0
     with pytest.raises(binding.TPMLPError):
-        binding.set_split_policy(3)
+        binding.set_split_policy(4)
 
 
 def _r256(x):
     return (x + 255) // 256 * 256
 
 
+# column sums of the bias gradients: ⌈T/128⌉·h for db; 2·⌈T/128⌉·F for da on
+# the tensor-core path (two partial rows per 128-row tile), ⌈T/128⌉·F on the
+# plain path
+def _colsums(T, h, F, tc=True):
+    c = -(-T // 128) if T > 0 else 1
+    return _r256(4 * c * h) + _r256(4 * (2 * c if tc else c) * F)
+
+
 def test_workspace_size_formula(lib):
-    """The workspace holds, each part rounded up to 256 bytes: the fp32 shard
-    partials S·T·h when the row products are split by shard, db's column-sum
-    partials ⌈T/128⌉·h, and da's: 2·⌈T/128⌉·F on the tensor-core path (two per
-    128-row tile when the GeLU′ epilogue sums them), ⌈T/128⌉·F on the plain path."""
+    """The workspace holds, each part rounded up to 256 bytes: the fp32 partial
+    tiles and the arrival counters of split tiles (none with whole tiles
+    only), then the bias gradients' column-sum partials."""
     import torch
     from tensor_transformer_mlp_block_b200 import binding
     binding.set_split_policy(1)
     try:
         for T, h, F, p in [(8192, 4096, 16384, 2), (300, 200, 520, 2), (1, 8, 8, 1), (129, 64, 264, 3)]:
-            c = -(-T // 128)
-            assert binding.workspace_size(T, h, F, p) == _r256(4 * c * h) + _r256(4 * 2 * c * F), (T, h, F)
-        assert binding.workspace_size(37, 12, 44, 2) == _r256(4 * 12) + _r256(4 * 44)  # plain path
+            assert binding.workspace_size(T, h, F, p) == _colsums(T, h, F), (T, h, F)
+        assert binding.workspace_size(37, 12, 44, 2) == _colsums(37, 12, 44, tc=False)  # plain path
         assert binding.workspace_size(512, 12, 48, 2, torch.float32) == _r256(16 * 12) + _r256(16 * 48)
         assert binding.workspace_size(0, 12, 44, 2) == _r256(4 * 12) + _r256(4 * 44)
         # the 7B-class step: 9 MiB
         assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20
-        binding.set_split_policy(2)  # split by shard: p planes of T·h fp32 in front
+        # one unit per shard and tile: 2 × 2 pair tiles of 256 × 256 fp32, p of
+        # each; 16 int counters per tile
+        binding.set_split_policy(2)
         T, h, F, p = 384, 320, 1024, 4
-        assert binding.workspace_size(T, h, F, p) == (_r256(4 * p * T * h) + _r256(4 * 3 * h)
-                                                      + _r256(4 * 6 * F))
+        tiles = 2 * 2
+        assert binding.workspace_size(T, h, F, p) == (_r256(tiles * p * 256 * 256 * 4)
+                                                      + _r256(tiles * 16 * 4) + _colsums(T, h, F))
+        # stream-K tail everywhere valid: two partial tiles and 16 counters per
+        # worker (74 CTA pairs of a 148-SM GPU); at 384 × 320 × 1024 no product
+        # has the 4 k-blocks per pair a tail needs
+        binding.set_split_policy(3)
+        assert binding.workspace_size(T, h, F, p) == _colsums(T, h, F)
+        T, h, F, p = 2048, 1024, 4096, 4
+        assert binding.plan_schedules(T, h, F, p)["F1"] == binding.SCHED_STREAMK
+        assert binding.workspace_size(T, h, F, p) == (_r256(2 * 74 * 256 * 256 * 4)
+                                                      + _r256(74 * 16 * 4) + _colsums(T, h, F))
     finally:
         binding.set_split_policy(0)
 
 
-def test_automatic_split_plan_for_the_named_workloads(lib):
-    """The automatic policy keeps the row products unsplit when the output
-    tiles fill the GPU (7B: 32 × 16 pair tiles over 74 pairs; GPT-2, 350M) and
-    splits them by shard when they do not (175B: 8 × 48 pair tiles over 74
-    pairs -> 2 shard groups). Seen through the workspace, which holds the
-    split planes. (Without a GPU the planner assumes 148 SMs.)"""
+def test_automatic_schedules_for_the_named_workloads(lib):
+    """The automatic policy keeps whole tiles where the last wave of 74 CTA
+    pairs is nearly full (every 7B-class product) or the tail would save less
+    than its own cost (GPT-2-small, 350M), and takes the stream-K tail for the
+    175B-class row-parallel products (8 × 48 pair tiles = 5.19 waves of
+    768 k-blocks). (Without a GPU the planner assumes 148 SMs.)"""
     from tensor_transformer_mlp_block_b200 import binding
     binding.set_split_policy(0)
-
-    def planes(T, h, F, p):
-        c = -(-T // 128)
-        extra = binding.workspace_size(T, h, F, p) - _r256(4 * c * h) - _r256(8 * c * F)
-        return extra / (4 * T * h)
-    assert planes(8192, 4096, 16384, 2) == 0
-    assert planes(4096, 768, 3072, 2) == 0
-    assert planes(6144, 1024, 4096, 4) == 0
-    assert planes(2048, 12288, 49152, 8) == 2
+    TILES, SK = binding.SCHED_TILES, binding.SCHED_STREAMK
+    assert set(binding.plan_schedules(8192, 4096, 16384, 2).values()) == {TILES}
+    assert binding.plan_schedules(2048, 12288, 49152, 8) == dict(F1=TILES, F2=SK, B2=TILES, B3=TILES,
+                                                                 B4=TILES, B5=SK)
+    assert set(binding.plan_schedules(4096, 768, 3072, 2).values()) == {TILES}
+    assert set(binding.plan_schedules(6144, 1024, 4096, 4).values()) == {TILES}
+    # policy 1: whole tiles everywhere; policy 2: shard groups for the row products
+    binding.set_split_policy(1)
+    assert set(binding.plan_schedules(2048, 12288, 49152, 8).values()) == {TILES}
+    binding.set_split_policy(2)
+    k = binding.plan_schedules(2048, 12288, 49152, 8)
+    assert k["F2"] == k["B5"] == binding.SCHED_GROUPS and k["F1"] == TILES
+    binding.set_split_policy(0)
 
 
 def test_product_path_refuses_cpu_tensors():

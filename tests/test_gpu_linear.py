@@ -80,7 +80,7 @@ def test_linear_plain_path_and_fp32(split):
     _check(_run(inp, 2, split), _oracle(inp), "fp32")
 
 
-@pytest.mark.parametrize("policy", [1, 2])
+@pytest.mark.parametrize("policy", [1, 2, 3])
 @pytest.mark.parametrize("split", ["columns", "rows"])
 def test_linear_shard_sum_schedules(policy, split):
     """Both schedules of the product that carries the shard sum (the forward

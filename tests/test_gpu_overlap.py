@@ -44,6 +44,7 @@ def _both(inp, p, act="gelu"):
     (384, 320, 1024, 4, 2, "gelu"),      # row products split by shard + ordered reduction
     (256, 128, 512, 4, 1, "gelu_tanh"),
     (37, 12, 44, 2, 0, "gelu"),          # plain kernels (ordinary launches)
+    (600, 3072, 1536, 2, 3, "gelu"),     # stream-K tail in every product
 ])
 def test_overlap_on_off_bit_identical(T, h, F, p, policy, act):
     binding.set_split_policy(policy)
@@ -61,7 +62,7 @@ def test_overlap_gpt2_full_oracle():
     compare_full(res[True], oracle_full(inp), "bf16")
 
 
-@pytest.mark.parametrize("policy", [0, 2])
+@pytest.mark.parametrize("policy", [0, 2, 3])
 def test_back_to_back_steps_on_shared_buffers(policy):
     """Five steps with new X and dZ each, all writing the same H, Y, Z and
     gradient buffers, queued without synchronising: each step's results

@@ -10,11 +10,17 @@ import numpy as np
 import pytest
 import torch
 
-from parity_util import TOL, compare_full, compare_sampled, oracle_full, rel_err, run_gpu, to_np
+from parity_util import (TOL, compare_full, compare_sampled, compare_to_sampled, oracle_full,
+                         oracle_sampled, rel_err, run_gpu, to_np)
 from tensor_transformer_mlp_block_b200 import configs
 from tensor_transformer_mlp_block_b200.inputs import make_inputs, make_shape, sample_indices
 
 pytestmark = pytest.mark.gpu
+
+
+# shard-sum schedules of tpmlp_set_split_policy: 0 automatic, 1 whole tiles
+# only, 2 every shard its own work unit, 3 stream-K tail wherever valid
+POLICIES = (0, 1, 2, 3)
 
 
 @pytest.fixture(autouse=True)
@@ -54,10 +60,11 @@ def test_bf16_unaligned_shape_plain_path():
     compare_full(gpu, oracle_full(inp), "bf16")
 
 
-@pytest.mark.parametrize("policy", [1, 2])
+@pytest.mark.parametrize("policy", [1, 2, 3])
 def test_row_parallel_split_policies(policy):
-    """Both schedules of the row-parallel products (shard K-loop in tensor
-    memory; per-shard fp32 partials summed in order) match the oracle."""
+    """Every schedule of the row-parallel products (shard K-loop in tensor
+    memory; per-shard fp32 partials summed in order; a stream-K tail) matches
+    the oracle."""
     from tensor_transformer_mlp_block_b200 import binding
     binding.set_split_policy(policy)
     inp = make_shape(384, 320, 1024, "bf16", seed_offset=11)
@@ -122,20 +129,53 @@ def test_nan_propagates_without_fault():
 def test_named_config_sampled(name):
     cfg = configs.get(name)
     inp = make_inputs(cfg)
-    gpu = run_gpu(inp, cfg.p)
-    n_rows = 16 if name == "175b" else 48
-    R = sample_indices(cfg.T, n_rows, seed=1234).numpy()
+    gpu = run_gpu(inp, cfg.p, keep_on_device=True)
+    R = sample_indices(cfg.T, 48, seed=1234).numpy()
     J = sample_indices(cfg.F, 64, seed=1235).numpy()
     errs = compare_sampled(gpu, inp, R, J, cfg.dtype)
     assert all(np.isfinite(list(errs.values())))
 
 
-def test_named_config_gpt2_full():
-    """The GPT-2-small MLP against the full oracle (every element)."""
-    cfg = configs.get("gpt2-small")
+@pytest.mark.parametrize("name", ["gpt2-small", "350m"])
+def test_named_config_full(name):
+    """The GPT-2-small and 350M-class MLPs against the full oracle (every
+    element of every output and gradient)."""
+    cfg = configs.get(name)
     inp = make_inputs(cfg)
     gpu = run_gpu(inp, cfg.p)
     compare_full(gpu, oracle_full(inp), "bf16")
+
+
+def test_shard_count_invariance_7b_sampled():
+    """The 7B-class workload with p = 1, 2, 4, 8 under every shard-sum
+    schedule: each matches the oracle on seeded rows and columns, and any two
+    agree element by element (every output, in full) within the same bound."""
+    from tensor_transformer_mlp_block_b200 import binding
+    cfg = configs.get("7b")
+    inp = make_inputs(cfg)
+    R = sample_indices(cfg.T, 16, seed=1234).numpy()
+    J = sample_indices(cfg.F, 32, seed=1235).numpy()
+    ref = oracle_sampled(inp, R, J)
+    base, rms = None, None
+    for policy in POLICIES:
+        binding.set_split_policy(policy)
+        for p in (1, 2, 4, 8):
+            out = run_gpu(inp, p, keep_on_device=True)
+            compare_to_sampled(out, ref, "bf16")
+            if base is None:
+                base = out
+                rms = {k: float(v.double().pow(2).mean().sqrt()) for k, v in base.items()}
+                continue
+            for k, v in out.items():
+                # outputs stored in bf16 are each rounded once: two results
+                # with different summation orders may round the same exact
+                # value to neighbouring bf16 numbers, up to u·|value| each
+                u = 2.0 ** -8 if v.dtype == torch.bfloat16 else 0.0
+                excess = (v.double() - base[k].double()).abs() - 2.0 * u * base[k].double().abs()
+                diff = float(excess.max())
+                assert diff <= TOL["bf16"] * rms[k], (policy, p, k, diff / rms[k])
+            del out
+    torch.cuda.empty_cache()
 
 
 @pytest.mark.parametrize("T,h,F,p", [(300, 200, 520, 2), (256, 128, 512, 4), (37, 12, 44, 2)])
@@ -213,7 +253,7 @@ def test_tensors_on_a_device_other_than_the_current_one():
         assert torch.equal(ref[k], got[k]), k
 
 
-@pytest.mark.parametrize("policy", [0, 2])
+@pytest.mark.parametrize("policy", [0, 2, 3])
 @pytest.mark.parametrize("T,h,F,p", [
     (200, 64, 64, 64),     # p = F: every shard is one hidden column
     (200, 64, 128, 16),    # Fp = 8: shards narrower than one 64-deep k-block
@@ -238,3 +278,40 @@ def test_fused_da_partials_at_tile_edges(T):
     inp = make_shape(T, 3072, 264, "bf16", seed_offset=T + 71)
     gpu = run_gpu(inp, 2)
     compare_full(gpu, oracle_full(inp), "bf16")
+
+
+@pytest.mark.parametrize("T,h,F,p", [
+    (600, 3072, 1536, 2),  # every product takes the tail; relaying GeLU / GeLU′ epilogues, da partials
+    (600, 512, 4096, 4),   # row products with the relaying bias epilogue (K = 4096)
+    (100, 3072, 8192, 2),  # one-CTA kernel (T ≤ 128): 148 workers, ragged rows
+    (1000, 1000, 2000, 2), # ragged M, N and K in the split tiles
+])
+def test_streamk_tail_full_oracle(T, h, F, p):
+    """Policy 3 (stream-K tail wherever valid): tiles split over CTA pairs at
+    arbitrary k-blocks, partials summed by the last unit to finish, against
+    the full oracle; two runs are bit-identical."""
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(3)
+    kinds = binding.plan_schedules(T, h, F, p)
+    assert binding.SCHED_STREAMK in kinds.values(), kinds
+    inp = make_shape(T, h, F, "bf16", seed_offset=T + h + 5)
+    a = run_gpu(inp, p)
+    compare_full(a, oracle_full(inp), "bf16")
+    b = run_gpu(inp, p)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+def test_streamk_tail_175b_row_products_sampled():
+    """The 175B-class workload as the automatic plan runs it (row-parallel
+    products on the stream-K tail) against the oracle on 48 seeded rows and
+    64 columns."""
+    from tensor_transformer_mlp_block_b200 import binding
+    cfg = configs.get("175b")
+    kinds = binding.plan_schedules(cfg.T, cfg.h, cfg.F, cfg.p)
+    assert kinds["F2"] == kinds["B5"] == binding.SCHED_STREAMK, kinds
+    inp = make_inputs(cfg)
+    gpu = run_gpu(inp, cfg.p, keep_on_device=True)
+    R = sample_indices(cfg.T, 48, seed=4321).numpy()
+    J = sample_indices(cfg.F, 64, seed=4322).numpy()
+    compare_sampled(gpu, inp, R, J, cfg.dtype)

@@ -26,7 +26,7 @@ def _cases(n=48, seed=2024):
             h = 8 * rng.randint(1, 48)
             Fp = 8 * rng.randint(1, 40)
         T = rng.choice([1, 2, 17, 64, 127, 128, 129, 255, 256, 257]) if i % 3 == 0 else rng.randint(1, 700)
-        out.append(dict(T=T, h=h, F=Fp * p, p=p, policy=rng.choice([0, 1, 2]),
+        out.append(dict(T=T, h=h, F=Fp * p, p=p, policy=rng.choice([0, 1, 2, 3]),
                         act=rng.choice(["gelu", "gelu_tanh"]), overlap=rng.random() < 0.7, seed=i))
     return out
 
@@ -60,7 +60,7 @@ def _linear_cases(n=24, seed=77):
             K = 8 * rng.randint(1, 40) * (p if split == "rows" else 1)
             N = 8 * rng.randint(1, 40) * (p if split == "columns" else 1)
         T = rng.choice([1, 2, 127, 128, 129, 256, 257]) if i % 3 == 0 else rng.randint(1, 600)
-        out.append(dict(T=T, K=K, N=N, p=p, split=split, policy=rng.choice([0, 1, 2]),
+        out.append(dict(T=T, K=K, N=N, p=p, split=split, policy=rng.choice([0, 1, 2, 3]),
                         overlap=rng.random() < 0.7, seed=i))
     return out
 

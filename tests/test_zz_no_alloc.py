@@ -41,6 +41,7 @@ def _noalloc(d, H, Y, out, T, h, F, p):
 
 @pytest.mark.parametrize("T,h,F,p,dtype", [
     (256, 768, 3072, 2, "bf16"),  # tp_mlp_bwd splits dX by shard here; this one never does
+    (300, 4096, 1024, 2, "bf16"), # h ≥ 3072: the relaying GeLU′ epilogue without da partials
     (300, 200, 520, 2, "bf16"),   # ragged tiles
     (37, 12, 44, 2, "bf16"),      # plain CUDA-core path
     (512, 12, 48, 2, "fp32"),     # the fp32 workload
@@ -59,7 +60,11 @@ def test_noalloc_backward_matches_backward_twice(T, h, F, p, dtype):
         torch.cuda.synchronize()
         assert binding.last_device_status() == binding.OK
         for k, r in ref.items():
-            err = rel_err(to_np(out[k]), r)
+            # dX and dH are stored in bf16 by both calls, each rounding once;
+            # where the two sum in different orders they may round the same
+            # value to neighbouring bf16 numbers (up to u·|value| each)
+            u = 2 * 2.0 ** -8 if out[k].dtype == torch.bfloat16 else 0.0
+            err = rel_err(to_np(out[k]), r, u)
             assert err <= TOL[dtype], (call, k, err)
 
 
