@@ -207,7 +207,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-i", str(self.gpu_index), "-lms", "100"],
+                 "-i", str(self.gpu_index), "-lms", "50"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
             self.proc = None
@@ -226,12 +226,15 @@ class ClockSampler:
                 if len(r) < 10:
                     continue
                 try:
-                    ts = time.mktime(time.strptime(r[0].strip().split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    stamp, _, frac = r[0].strip().partition(".")
+                    ts = time.mktime(time.strptime(stamp, "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + frac) if frac.isdigit() else 0.0
                     rows.append((ts, [c.strip() for c in r]))
                 except Exception:
                     continue
         os.unlink(self.path)
-        inside = [c for ts, c in rows if t0 - 1.0 <= ts <= t1 + 1.0] or [c for _, c in rows]
+        # samples taken while the timed work ran
+        inside = [c for ts, c in rows if t0 <= ts <= t1] or [c for _, c in rows]
         if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
         sm = [float(c[2]) for c in inside if c[2].replace(".", "").isdigit()]

@@ -85,8 +85,13 @@ struct GemmArgs {
     // Tiles split over several units (SCHED_GROUPS, the stream-K tail):
     // fp32 partial tiles (partial_chunk) and 16 arrival counters per split
     // tile (one per CTA of the pair and epilogue warp), all zero at launch.
+    // (colsum_out must be null: a split tile is finished warp by warp.)
     float* partials;
     int* counters;
+    // Counters of a later launch on the same stream, zeroed by this one
+    // (which must not split tiles itself): zero_count ints at zero_counters.
+    int* zero_counters;
+    int zero_count;
 };
 
 constexpr int kBM = 128;
@@ -262,32 +267,24 @@ __device__ __forceinline__ void partial_store(float* chunk, const uint32_t (&acc
 }
 
 // acc = Σ_{q = 0 .. pieces-1} partial q, added in ascending q (ascending k).
+// (The partials sit in L2, written by other SMs: each piece costs one round
+// trip, with this lane's 8 loads of it in flight together.)
 __device__ __forceinline__ void partial_sum(const GemmArgs& g, const WorkUnit& w, int nworkers,
                                             int tile_rows, int bn, int r0, int c0,
                                             uint32_t (&acc)[32], int lane) {
-    {
-        const float4* p = reinterpret_cast<const float4*>(
-            partial_chunk(g, partial_slot(g, w, 0, nworkers), tile_rows, bn, r0, c0));
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float4 x = __ldcg(p + 32 * j + lane);
-            acc[4 * j] = __float_as_uint(x.x);
-            acc[4 * j + 1] = __float_as_uint(x.y);
-            acc[4 * j + 2] = __float_as_uint(x.z);
-            acc[4 * j + 3] = __float_as_uint(x.w);
-        }
-    }
 #pragma unroll 1
-    for (int q = 1; q < w.pieces; ++q) {
+    for (int q = 0; q < w.pieces; ++q) {
         const float4* p = reinterpret_cast<const float4*>(
             partial_chunk(g, partial_slot(g, w, q, nworkers), tile_rows, bn, r0, c0));
+        float4 x[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) x[j] = __ldcg(p + 32 * j + lane);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 x = __ldcg(p + 32 * j + lane);
-            acc[4 * j] = __float_as_uint(__uint_as_float(acc[4 * j]) + x.x);
-            acc[4 * j + 1] = __float_as_uint(__uint_as_float(acc[4 * j + 1]) + x.y);
-            acc[4 * j + 2] = __float_as_uint(__uint_as_float(acc[4 * j + 2]) + x.z);
-            acc[4 * j + 3] = __float_as_uint(__uint_as_float(acc[4 * j + 3]) + x.w);
+            const float v[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+                acc[4 * j + e] = __float_as_uint(q == 0 ? v[e] : __uint_as_float(acc[4 * j + e]) + v[e]);
         }
     }
 }
@@ -628,6 +625,13 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
 // full/empty mbarrier pair per relay (bounded waits). Relaying doubles the
 // work of the computing warps, so it pays only when a tile's main loop is
 // long enough to hide it; the host picks the instantiation per launch.
+// Whether an instantiation can finish split tiles. The relaying GeLU′
+// epilogue sums da's columns over the rows of two warps, which a split tile
+// (finished warp by warp) does not have together: its launches always run
+// whole tiles (the host keeps them so), and the split path is compiled out.
+template <int EPI, bool RELAY>
+constexpr bool kSplittable = !(EpiTraits<EPI>::kDAct && RELAY);
+
 template <int BN, int EPI, bool PAIR, bool RELAY>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
                                               const CUtensorMap* tmO1, uint32_t tmem_base,
@@ -650,6 +654,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         if (EpiTraits<EPI>::kAct) tma_prefetch_desc(tmO1);
     }
     uint32_t xcount = 0;
+    bool stored = false;  // a relay warp has bulk stores of a split tile in flight
     WorkIter it = work_iter(worker, nworkers);
     WorkUnit w;
     for (int local = 0; next_unit(g, it, w); ++local) {
@@ -666,12 +671,54 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         const int tile_row0 = w.mb * tile_rows + cta_row_off;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                static_cast<uint32_t>(buf * BN);
-        // a split tile: this unit writes its partial; the last to arrive sums
-        const bool split = w.pieces > 1;
-        const int64_t my_slot = split ? partial_slot(g, w, w.piece, nworkers) : 0;
-        // rows of this warp's own chunks and of the relayed ones, within the tile
-        const int own_r = cta_row_off + quad * 32;
-        const int rel_r = cta_row_off + (quad - 2) * 32;
+        if (kSplittable<EPI, RELAY> && w.pieces > 1) {
+            // A split tile. Every epilogue warp (no relay) takes its own 32
+            // rows and half of the columns: it stores its fp32 partial, and
+            // the warp of the last unit to arrive adds the tile's partials in
+            // ascending k order and runs the epilogue for those rows.
+            const int64_t my_slot = partial_slot(g, w, w.piece, nworkers);
+            const int own_r = cta_row_off + quad * 32;
+#pragma unroll 1
+            for (int i = 0; i < kChunks; ++i) {
+                const int c = half * kChunks + i;
+                uint32_t acc[32];
+                tmem_ld_32x32b_x32(t_row + c * 32, acc);
+                tmem_wait_ld();
+                if (i == kChunks - 1) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) {
+                        if constexpr (PAIR)
+                            mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+                        else
+                            mbar_arrive(smem_u32(&tempty[buf]));
+                    }
+                }
+                partial_store(partial_chunk(g, my_slot, tile_rows, BN, own_r, c * 32), acc, lane);
+            }
+            // one counter per split tile, CTA of the pair and epilogue warp
+            int* ctr = g.counters + (static_cast<int64_t>(w.key) * 2 + cta_row_off / kBM) * 8 + (warp - 2);
+            if (partial_arrive(ctr, w.pieces, lane)) {
+                float csx[32];  // unused: no column sums on split tiles
+#pragma unroll 1
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c = half * kChunks + i;
+                    uint32_t acc[32];
+                    partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane);
+                    epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, w.nb * BN + c * 32,
+                                        slot, lane, csx, 0, -1);
+                }
+                stored = true;
+            }
+            continue;
+        }
+        if (RELAY && relay && stored) {
+            // the slot becomes a hand-off buffer again: the split tile's bulk
+            // stores must have finished reading it
+            if (lane == 0) bulk_wait_read0();
+            __syncwarp();
+            stored = false;
+        }
         bool failed = false;
         float csx[32];  // da partial of the current columns (relay, GeLU′ only)
         // da partials (relay only): the own rows and the partner's rows of these
@@ -712,11 +759,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 ++xcount;
                 continue;
             }
-            if (split)
-                partial_store(partial_chunk(g, my_slot, tile_rows, BN, own_r, c * 32), acc, lane);
-            else
-                epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane, csx,
-                                    cs_on ? 1 : 0, cs_row);
+            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane, csx,
+                                cs_on ? 1 : 0, cs_row);
             if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
                 const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
@@ -735,40 +779,24 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 }
                 mbar_arrive(smem_u32(&xempty[pair_id]));
                 ++xcount;
-                if (split)
-                    partial_store(partial_chunk(g, my_slot, tile_rows, BN, rel_r, c * 32), pacc, lane);
-                else
-                    epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, slot,
-                                        lane, csx, cs_on ? 2 : 0, cs_row);
+                epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, slot, lane,
+                                    csx, cs_on ? 2 : 0, cs_row);
             }
         }
         if (failed) {
             raise_timeout(abort);
             break;
         }
-        if (split && !(RELAY && relay)) {
-            // one counter per split tile, CTA of the pair and epilogue warp
-            int* ctr = g.counters + (static_cast<int64_t>(w.key) * 2 + cta_row_off / kBM) * 8 + (warp - 2);
-            if (partial_arrive(ctr, w.pieces, lane)) {
-#pragma unroll 1
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c = half * kChunks + i;
-                    const int col0 = w.nb * BN + c * 32;
-                    uint32_t acc[32];
-                    partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane);
-                    epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane,
-                                        csx, cs_on ? 1 : 0, cs_row);
-                    if constexpr (RELAY) {
-                        partial_sum(g, w, nworkers, tile_rows, BN, rel_r, c * 32, acc, lane);
-                        epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + (quad - 2) * 32, col0,
-                                            slot, lane, csx, cs_on ? 2 : 0, cs_row);
-                    }
-                }
-            }
-        }
     }
-    if (lane == 0 && !relay) bulk_wait0();  // this warp's stores are complete before exit
+    if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
     __syncwarp();
+}
+
+// Counters of a later launch (GemmArgs::zero_counters), zeroed by the idle
+// lanes of warp 0 of every CTA after the wait for the predecessor.
+__device__ __forceinline__ void zero_later_counters(const GemmArgs& g, int lane) {
+    if (g.zero_counters == nullptr || lane == 0) return;
+    for (int i = blockIdx.x * 31 + lane - 1; i < g.zero_count; i += gridDim.x * 31) g.zero_counters[i] = 0;
 }
 
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
@@ -831,6 +859,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     grid_dep_launch();
 
     const uint64_t limit = g.wait_limit_ns;
+    if (warp == 0) zero_later_counters(g, lane);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer

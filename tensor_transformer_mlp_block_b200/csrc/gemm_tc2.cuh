@@ -100,6 +100,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     grid_dep_launch();
 
     const uint64_t limit = g.wait_limit_ns;  // num_m_blocks counts 256-row blocks
+    if (warp == 0) zero_later_counters(g, lane);
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)

@@ -278,13 +278,15 @@ bool streamk_pays(int64_t tiles, int64_t kb, int64_t P, bool force) {
 }
 
 // Fill g's schedule for at most P workers; returns the number of workers
-// to launch. A split schedule needs the partial-tile workspace.
-int resolve_sched(GemmArgs& g, const SchedReq& req, int64_t P) {
+// to launch. A split schedule needs the partial-tile workspace, a kernel
+// instantiation that can finish split tiles, and no column-sum output.
+int resolve_sched(GemmArgs& g, const SchedReq& req, int64_t P, bool splittable) {
     const int64_t tiles = static_cast<int64_t>(g.num_m_blocks) * g.num_n_blocks;
     g.sched = SCHED_TILES;
     g.groups = 1;
     g.kb_per_group = g.k_blocks;
-    const bool have_ws = g.partials != nullptr && g.counters != nullptr;
+    const bool have_ws = g.partials != nullptr && g.counters != nullptr && splittable &&
+                         g.colsum_out == nullptr;
     if (req.kind == SCHED_GROUPS && have_ws && req.groups > 1 && g.k_blocks % req.groups == 0) {
         g.sched = SCHED_GROUPS;
         g.groups = req.groups;
@@ -332,7 +334,7 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
             g_dev[devn].attr_set |= uint64_t(1) << id;
         }
     }
-    const int grid = resolve_sched(g, req, dev->num_sms);
+    const int grid = resolve_sched(g, req, dev->num_sms, kSplittable<EPI, RELAY>);
     return launch_dep(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1, g);
 }
 
@@ -387,7 +389,7 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
         max_pairs = d.max_pairs[id];
     }
     // never more workers than the plan sized the workspace for (num_sms / 2)
-    const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2));
+    const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2), kSplittable<EPI, RELAY>);
     return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
                       g);
 }
@@ -480,9 +482,10 @@ struct SplitSpace {
 // The geometry is the launcher's: CTA pairs with 256-row tiles and
 // num_sms / 2 workers when M > 128, else one CTA per 128-row tile and
 // num_sms workers; 256-column tiles.
-SchedReq plan_sched(int64_t M, int64_t N, int64_t K, int shard_groups, int num_sms, SplitSpace* sp) {
+SchedReq plan_sched(int64_t M, int64_t N, int64_t K, int shard_groups, int num_sms, SplitSpace* sp,
+                    bool may_split = true) {
     SchedReq r;
-    const int policy = g_split_policy.load();
+    const int policy = may_split ? g_split_policy.load() : 1;
     const bool pairs = M > kBM;
     const int64_t tile_rows = pairs ? kPairM : kBM;
     const int64_t workers = pairs ? num_sms / 2 : num_sms;
@@ -533,7 +536,10 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
         const int sms = plan_num_sms();
         pl->f1 = plan_sched(T, F, h, 0, sms, &sp);                   // X·A
         pl->f2 = plan_sched(T, h, F, shard_groups(F, p), sms, &sp);  // Σ Y_i·B_i
-        pl->b2 = plan_sched(T, F, h, 0, sms, &sp);                   // dZ·Bᵀ
+        // dZ·Bᵀ: whole tiles when its relaying epilogue also sums da's columns
+        // (those sums pair the rows of two warps, which a split tile, finished
+        // warp by warp, does not have together)
+        pl->b2 = plan_sched(T, F, h, 0, sms, &sp, h < kRelayMinKAct);
         pl->b3 = plan_sched(F, h, T, 0, sms, &sp);                   // Yᵀ·dZ
         pl->b4 = plan_sched(h, F, T, 0, sms, &sp);                   // Xᵀ·dH
         pl->b5 = plan_sched(T, h, F, shard_groups(F, p), sms, &sp);  // Σ dH_i·A_iᵀ
@@ -650,6 +656,20 @@ tpmlp_status reset_counters(void* workspace, size_t off, size_t bytes, cudaStrea
 void set_split_space(GemmArgs& g, void* workspace, size_t off_part, size_t off_ctr) {
     g.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + off_part);
     g.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + off_ctr);
+}
+
+// The counters must be zero before the first product of a call that splits
+// tiles. `g` is the call's first GEMM (launched next, with schedule `req`):
+// if it runs whole tiles, its own kernel zeroes them for the later products
+// (no extra launch); otherwise a reset kernel runs first.
+tpmlp_status zero_counters_before(GemmArgs& g, const SchedReq& req, void* workspace, size_t off_ctr,
+                                  size_t bytes, cudaStream_t st) {
+    if (req.kind == SCHED_TILES) {
+        g.zero_counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + off_ctr);
+        g.zero_count = static_cast<int>(bytes / sizeof(int));
+        return TPMLP_OK;
+    }
+    return reset_counters(workspace, off_ctr, bytes, st);
 }
 
 #define TPMLP_TRY(expr)                         \
@@ -774,11 +794,11 @@ tpmlp_status linear_bwd_impl(const void* dY, const void* X, const void* W, void*
         for (const void* q : {dY, X, W, static_cast<const void*>(dX), static_cast<const void*>(dW),
                               static_cast<const void*>(dbias)})
             if (!aligned16(q)) return TPMLP_ERR_ALIGN;
-        if (pl.bwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         TPMLP_TRY(colsum(K_L_DB, static_cast<const __nv_bfloat16*>(dY), T, N, pl.chunks, cs, dbias, st));
         // dW = Xᵀ·dY: Aop = X [T][K] (MN-major, M = K), Bop = dY [T][N] (MN-major)
         GemmArgs gw{};
         set_split_space(gw, workspace, pl.off_part, pl.off_ctr);
+        if (pl.bwd_split) TPMLP_TRY(zero_counters_before(gw, pl.dw, workspace, pl.off_ctr, pl.ctr_bytes, st));
         gw.out0 = dW;
         gw.ld_out = N;
         TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_L_DW, X, dY, iK, iN, iT, pl.dw, gw, st)));
@@ -833,10 +853,11 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
         const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
         // without F2 (activation recompute) there is no workspace: whole tiles
         const SchedReq f1 = with_f2 ? pl.f1 : SchedReq{};
-        if (with_f2 && pl.fwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         // F1: H = X·A + a, Y = GeLU(H). Aop = X [T][h] (K-major), Bop = A [h][F] (MN-major).
         GemmArgs g1{};
         if (with_f2) set_split_space(g1, workspace, pl.off_part, pl.off_ctr);
+        if (with_f2 && pl.fwd_split)
+            TPMLP_TRY(zero_counters_before(g1, f1, workspace, pl.off_ctr, pl.ctr_bytes, st));
         g1.out0 = H;
         g1.out1 = Y;
         g1.ld_out = F;
@@ -905,7 +926,6 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
             if (!aligned16(q)) return TPMLP_ERR_ALIGN;
         const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
         const __nv_bfloat16* dZb = static_cast<const __nv_bfloat16*>(dZ);
-        if (pl.bwd_split) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         // db = 1ᵀ·dZ
         TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
@@ -916,6 +936,7 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         const bool fused_da = h >= kRelayMinKAct;
         GemmArgs g2{};
         set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
+        if (pl.bwd_split) TPMLP_TRY(zero_counters_before(g2, pl.b2, workspace, pl.off_ctr, pl.ctr_bytes, st));
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
