@@ -92,6 +92,11 @@ struct GemmArgs {
     // (which must not split tiles itself): zero_count ints at zero_counters.
     int* zero_counters;
     int zero_count;
+    // A second product in the same launch (CTA-pair kernel, whole tiles, same
+    // K and fp32 epilogue; operands in tmA2 / tmB2, output in tmO1): its
+    // M2 × N2 tiles follow the first product's. second = 0: none.
+    int second;
+    int M2, N2, num_m_blocks2, num_n_blocks2;
 };
 
 constexpr int kBM = 128;
@@ -123,18 +128,23 @@ struct TileCfg {
 
 // Output tile t in grouped raster order: kGroupM m-blocks per group,
 // m fastest inside a group, so that neighbouring units share Bop panels.
-TPMLP_HD void tile_coords(const GemmArgs& g, int t, int& mb, int& nb) {
-    const int per_group = kGroupM * g.num_n_blocks;
+TPMLP_HD void tile_coords_of(int num_m_blocks, int num_n_blocks, int t, int& mb, int& nb) {
+    const int per_group = kGroupM * num_n_blocks;
     const int group = t / per_group;
     const int first_m = group * kGroupM;
-    const int rem_m = g.num_m_blocks - first_m;
+    const int rem_m = num_m_blocks - first_m;
     const int gm = rem_m < kGroupM ? rem_m : kGroupM;
     const int idx = t - group * per_group;
     mb = first_m + idx % gm;
     nb = idx / gm;
 }
 
+TPMLP_HD void tile_coords(const GemmArgs& g, int t, int& mb, int& nb) {
+    tile_coords_of(g.num_m_blocks, g.num_n_blocks, t, mb, nb);
+}
+
 struct WorkUnit {
+    int prob;      // 0, or 1 for the second product of a grouped launch
     int mb, nb;    // output tile
     int kb0, kb1;  // k-blocks [kb0, kb1) of this unit
     int pieces;    // units sharing the tile (1: the whole K range)
@@ -188,6 +198,7 @@ TPMLP_HD bool next_unit(const GemmArgs& g, WorkIter& it, WorkUnit& w) {
         const int s = u / tiles;
         const int t = u - s * tiles;
         tile_coords(g, t, w.mb, w.nb);
+        w.prob = 0;
         w.kb0 = s * g.kb_per_group;
         w.kb1 = w.kb0 + g.kb_per_group < g.k_blocks ? w.kb0 + g.kb_per_group : g.k_blocks;
         w.pieces = g.groups;
@@ -199,9 +210,14 @@ TPMLP_HD bool next_unit(const GemmArgs& g, WorkIter& it, WorkUnit& w) {
     const int whole = g.sched == SCHED_STREAMK ? sk_whole_tiles(g, it.nworkers) : tiles;
     if (!it.tail) {
         const int u = it.worker + it.next * it.nworkers;
-        if (u < whole) {
+        const int tiles2 = (g.second && g.sched == SCHED_TILES) ? g.num_m_blocks2 * g.num_n_blocks2 : 0;
+        if (u < whole + tiles2) {
             ++it.next;
-            tile_coords(g, u, w.mb, w.nb);
+            w.prob = u < whole ? 0 : 1;
+            if (w.prob == 0)
+                tile_coords(g, u, w.mb, w.nb);
+            else
+                tile_coords_of(g.num_m_blocks2, g.num_n_blocks2, u - whole, w.mb, w.nb);
             w.kb0 = 0;
             w.kb1 = g.k_blocks;
             w.pieces = 1;
@@ -225,6 +241,7 @@ TPMLP_HD bool next_unit(const GemmArgs& g, WorkIter& it, WorkUnit& w) {
     const int64_t room = w.kb0 + (it.end - it.cur);
     w.kb1 = static_cast<int>(room < kb ? room : kb);
     tile_coords(g, whole + st, w.mb, w.nb);
+    w.prob = 0;
     w.seg_lo = sk_seg_of(first, W, it.nworkers);
     w.pieces = sk_seg_of(first + kb - 1, W, it.nworkers) - w.seg_lo + 1;
     w.piece = it.worker - w.seg_lo;
@@ -267,26 +284,42 @@ __device__ __forceinline__ void partial_store(float* chunk, const uint32_t (&acc
 }
 
 // acc = Σ_{q = 0 .. pieces-1} partial q, added in ascending q (ascending k).
-// (The partials sit in L2, written by other SMs: each piece costs one round
-// trip, with this lane's 8 loads of it in flight together.)
+// The partials sit in L2, written by other SMs (one round trip per piece, its
+// 8 loads per lane in flight together). Piece own_q (if ≥ 0) is this unit's
+// own, still in tensor memory at t_chunk: it is read from there at its place
+// in the order, so the sum is the same as from memory.
 __device__ __forceinline__ void partial_sum(const GemmArgs& g, const WorkUnit& w, int nworkers,
                                             int tile_rows, int bn, int r0, int c0,
-                                            uint32_t (&acc)[32], int lane) {
+                                            uint32_t (&acc)[32], int lane, int own_q,
+                                            uint32_t t_chunk) {
 #pragma unroll 1
     for (int q = 0; q < w.pieces; ++q) {
-        const float4* p = reinterpret_cast<const float4*>(
-            partial_chunk(g, partial_slot(g, w, q, nworkers), tile_rows, bn, r0, c0));
-        float4 x[8];
+        uint32_t x[32];
+        if (q == own_q) {
+            tmem_ld_32x32b_x32(t_chunk, x);
+            tmem_wait_ld();
+        } else {
+            const uint4* p = reinterpret_cast<const uint4*>(
+                partial_chunk(g, partial_slot(g, w, q, nworkers), tile_rows, bn, r0, c0));
 #pragma unroll
-        for (int j = 0; j < 8; ++j) x[j] = __ldcg(p + 32 * j + lane);
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-            const float v[4] = {x[j].x, x[j].y, x[j].z, x[j].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-                acc[4 * j + e] = __float_as_uint(q == 0 ? v[e] : __uint_as_float(acc[4 * j + e]) + v[e]);
+            for (int j = 0; j < 8; ++j) {
+                const uint4 v = __ldcg(p + 32 * j + lane);
+                x[4 * j] = v.x;
+                x[4 * j + 1] = v.y;
+                x[4 * j + 2] = v.z;
+                x[4 * j + 3] = v.w;
+            }
         }
+#pragma unroll
+        for (int i = 0; i < 32; ++i)
+            acc[i] = q == 0 ? x[i] : __float_as_uint(__uint_as_float(acc[i]) + __uint_as_float(x[i]));
     }
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
 }
 
 // Arrival of one epilogue warp on its counter of a split tile, after
@@ -512,11 +545,11 @@ template <int EPI>
 // and write the column sums to colsum_out row cs_row (if cs_row ≥ 0).
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensorMap* tmO0,
                                                const CUtensorMap* tmO1, const uint32_t (&acc)[32],
-                                               int row0, int col0, uint32_t slot,
+                                               int row0, int col0, int M, int N, uint32_t slot,
                                                int lane, float (&csx)[32], int cs_mode,
                                                int64_t cs_row) {
     const int row = row0 + lane;
-    const bool any = (row0 < g.M) && (col0 < g.N);
+    const bool any = (row0 < M) && (col0 < N);
     if constexpr (EPI == EPI_F32) {
         if (lane == 0) bulk_wait_read0();
         __syncwarp();
@@ -541,7 +574,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
 #pragma unroll
             for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(acc[8 * q + i]);
             if constexpr (EpiTraits<EPI>::kBias) {
-                if (g.bias != nullptr && c < g.N) {
+                if (g.bias != nullptr && c < N) {
                     float bb[8];
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.bias + c)), bb);
 #pragma unroll
@@ -550,7 +583,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             }
             if constexpr (EpiTraits<EPI>::kDAct) {
                 float hh[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-                if (row < g.M && c < g.N)
+                if (row < M && c < N)
                     unpack_bf16x8(__ldg(reinterpret_cast<const uint4*>(g.aux + off + 8 * q)), hh);
 #pragma unroll
                 for (int i = 0; i < 8; i += 2) {
@@ -602,7 +635,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
                 }
                 if (cs_mode == 2) {
                     const float s = warp_column_sums32(csx, lane);
-                    if (cs_row >= 0 && col0 + lane < g.N) g.colsum_out[cs_row * g.N + col0 + lane] = s;
+                    if (cs_row >= 0 && col0 + lane < N) g.colsum_out[cs_row * N + col0 + lane] = s;
                 }
             }
         }
@@ -627,10 +660,12 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
 // long enough to hide it; the host picks the instantiation per launch.
 // Whether an instantiation can finish split tiles. The relaying GeLU′
 // epilogue sums da's columns over the rows of two warps, which a split tile
-// (finished warp by warp) does not have together: its launches always run
-// whole tiles (the host keeps them so), and the split path is compiled out.
+// (finished warp by warp) does not have together; the relaying GeLU epilogue
+// has no registers to spare for the split path (it would spill in the
+// whole-tile path too). Their launches always run whole tiles (the host keeps
+// them so), and the split path is compiled out of them.
 template <int EPI, bool RELAY>
-constexpr bool kSplittable = !(EpiTraits<EPI>::kDAct && RELAY);
+constexpr bool kSplittable = !((EpiTraits<EPI>::kDAct || EpiTraits<EPI>::kAct) && RELAY);
 
 template <int BN, int EPI, bool PAIR, bool RELAY>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
@@ -651,7 +686,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     const uint32_t partner_slot = smem_u32(sEpi + (4 * half + quad) * kEpiSlotBytes);
     if (lane == 0 && !relay) {
         tma_prefetch_desc(tmO0);
-        if (EpiTraits<EPI>::kAct) tma_prefetch_desc(tmO1);
+        if (EpiTraits<EPI>::kAct || g.second) tma_prefetch_desc(tmO1);
     }
     uint32_t xcount = 0;
     bool stored = false;  // a relay warp has bulk stores of a split tile in flight
@@ -671,20 +706,63 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         const int tile_row0 = w.mb * tile_rows + cta_row_off;
         const uint32_t t_row = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
                                static_cast<uint32_t>(buf * BN);
+        // the unit's product: sizes and output map (a grouped launch's second
+        // product stores through tmO1; grouping is for single-output epilogues)
+        const int uM = w.prob ? g.M2 : g.M;
+        const int uN = w.prob ? g.N2 : g.N;
+        const CUtensorMap* uO = w.prob ? tmO1 : tmO0;
         if (kSplittable<EPI, RELAY> && w.pieces > 1) {
             // A split tile. Every epilogue warp (no relay) takes its own 32
-            // rows and half of the columns: it stores its fp32 partial, and
-            // the warp of the last unit to arrive adds the tile's partials in
-            // ascending k order and runs the epilogue for those rows.
-            const int64_t my_slot = partial_slot(g, w, w.piece, nworkers);
+            // rows and half of the columns; the warp of the last unit to arrive
+            // adds the tile's partials in ascending k order and runs the
+            // epilogue for those rows.
             const int own_r = cta_row_off + quad * 32;
+            // one counter per split tile, CTA of the pair and epilogue warp
+            int* ctr = g.counters + (static_cast<int64_t>(w.key) * 2 + cta_row_off / kBM) * 8 + (warp - 2);
+            // If every other unit of the tile has arrived already, this one is
+            // the last for certain: it neither stores its partial nor arrives,
+            // and takes its own part from tensor memory while summing.
+            int seen = 0;
+            if (lane == 0) seen = ld_acquire_gpu(ctr);
+            seen = __shfl_sync(0xffffffffu, seen, 0);
+            const bool sure_last = (seen == w.pieces - 1);
+            bool last = sure_last;
+            if (!sure_last) {
+                const int64_t my_slot = partial_slot(g, w, w.piece, nworkers);
 #pragma unroll 1
-            for (int i = 0; i < kChunks; ++i) {
-                const int c = half * kChunks + i;
-                uint32_t acc[32];
-                tmem_ld_32x32b_x32(t_row + c * 32, acc);
-                tmem_wait_ld();
-                if (i == kChunks - 1) {
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c = half * kChunks + i;
+                    uint32_t acc[32];
+                    tmem_ld_32x32b_x32(t_row + c * 32, acc);
+                    tmem_wait_ld();
+                    if (i == kChunks - 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) {
+                            if constexpr (PAIR)
+                                mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
+                            else
+                                mbar_arrive(smem_u32(&tempty[buf]));
+                        }
+                    }
+                    partial_store(partial_chunk(g, my_slot, tile_rows, BN, own_r, c * 32), acc, lane);
+                }
+                last = partial_arrive(ctr, w.pieces, lane);
+            }
+            if (last) {
+                float csx[32];  // unused: no column sums on split tiles
+#pragma unroll 1
+                for (int i = 0; i < kChunks; ++i) {
+                    const int c = half * kChunks + i;
+                    uint32_t acc[32];
+                    partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane,
+                                sure_last ? w.piece : -1, t_row + c * 32);
+                    epilogue_chunk<EPI>(g, uO, tmO1, acc, tile_row0 + quad * 32, w.nb * BN + c * 32,
+                                        uM, uN, slot, lane, csx, 0, -1);
+                }
+                if (sure_last) {
+                    // the accumulator was read in the loop above: release it, and
+                    // put the counter (at pieces - 1) back to zero
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) {
@@ -692,21 +770,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                             mbar_arrive_cluster(mapa_shared(smem_u32(&tempty[buf]), 0));
                         else
                             mbar_arrive(smem_u32(&tempty[buf]));
+                        atomicExch(ctr, 0);
                     }
-                }
-                partial_store(partial_chunk(g, my_slot, tile_rows, BN, own_r, c * 32), acc, lane);
-            }
-            // one counter per split tile, CTA of the pair and epilogue warp
-            int* ctr = g.counters + (static_cast<int64_t>(w.key) * 2 + cta_row_off / kBM) * 8 + (warp - 2);
-            if (partial_arrive(ctr, w.pieces, lane)) {
-                float csx[32];  // unused: no column sums on split tiles
-#pragma unroll 1
-                for (int i = 0; i < kChunks; ++i) {
-                    const int c = half * kChunks + i;
-                    uint32_t acc[32];
-                    partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane);
-                    epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, w.nb * BN + c * 32,
-                                        slot, lane, csx, 0, -1);
                 }
                 stored = true;
             }
@@ -725,7 +790,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
         // columns form one row of colsum_out per computing warp and CTA tile
         const bool cs_on = RELAY && g.colsum_out != nullptr;
         const int64_t cs_row =
-            tile_row0 < g.M ? static_cast<int64_t>(tile_row0 / kBM) * 2 + (quad - 2) : -1;
+            tile_row0 < uM ? static_cast<int64_t>(tile_row0 / kBM) * 2 + (quad - 2) : -1;
 #pragma unroll 1
         for (int i = 0; i < kChunks; ++i) {
             const int c = half * kChunks + i;
@@ -759,7 +824,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 ++xcount;
                 continue;
             }
-            epilogue_chunk<EPI>(g, tmO0, tmO1, acc, tile_row0 + quad * 32, col0, slot, lane, csx,
+            epilogue_chunk<EPI>(g, uO, tmO1, acc, tile_row0 + quad * 32, col0, uM, uN, slot, lane, csx,
                                 cs_on ? 1 : 0, cs_row);
             if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
@@ -779,8 +844,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 }
                 mbar_arrive(smem_u32(&xempty[pair_id]));
                 ++xcount;
-                epilogue_chunk<EPI>(g, tmO0, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, slot, lane,
-                                    csx, cs_on ? 2 : 0, cs_row);
+                epilogue_chunk<EPI>(g, uO, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, uM, uN, slot,
+                                    lane, csx, cs_on ? 2 : 0, cs_row);
             }
         }
         if (failed) {

@@ -40,6 +40,7 @@ template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
+                    const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs g) {
     using C = Tile2Cfg<BN>;
     constexpr int STAGES = C::STAGES;
@@ -107,6 +108,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tmA);
             tma_prefetch_desc(&tmB);
+            if (g.second) {
+                tma_prefetch_desc(&tmA2);
+                tma_prefetch_desc(&tmB2);
+            }
             int stage = 0;
             uint32_t phase = 0;
             int issued = 0;
@@ -118,6 +123,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             while (ok && next_unit(g, it, w)) {
                 const int mb = w.mb, nb = w.nb;
                 const int kb0 = w.kb0, kb1 = w.kb1;
+                const CUtensorMap* mA = w.prob ? &tmA2 : &tmA;
+                const CUtensorMap* mB = w.prob ? &tmB2 : &tmB;
                 for (int kb = kb0; kb < kb1; ++kb) {
                     if (!mbar_wait_bounded(smem_u32(&empty[stage]), phase ^ 1u, abort, limit)) {
                         raise_timeout(abort);
@@ -132,17 +139,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                     const int m0 = mb * kPairM + a_row0;
                     const int n0 = nb * BN + b_col0;
                     if constexpr (!A_MN) {
-                        tma_load_2d_pair(a_dst, &tmA, fb, kb * kBK, m0);
+                        tma_load_2d_pair(a_dst, mA, fb, kb * kBK, m0);
                     } else {
-                        tma_load_2d_pair(a_dst, &tmA, fb, m0, kb * kBK);
-                        tma_load_2d_pair(a_dst + 8192, &tmA, fb, m0 + 64, kb * kBK);
+                        tma_load_2d_pair(a_dst, mA, fb, m0, kb * kBK);
+                        tma_load_2d_pair(a_dst + 8192, mA, fb, m0 + 64, kb * kBK);
                     }
                     if constexpr (!B_MN) {
-                        tma_load_2d_pair(b_dst, &tmB, fb, kb * kBK, n0);
+                        tma_load_2d_pair(b_dst, mB, fb, kb * kBK, n0);
                     } else {
 #pragma unroll
                         for (int j = 0; j < BN / 128; ++j)
-                            tma_load_2d_pair(b_dst + j * 8192, &tmB, fb, n0 + j * 64, kb * kBK);
+                            tma_load_2d_pair(b_dst + j * 8192, mB, fb, n0 + j * 64, kb * kBK);
                     }
                     ++issued;
                     if (++stage == STAGES) {

@@ -172,13 +172,13 @@ tpmlp_status launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 // ------------------------------------------------------- per-kernel timing
 
 enum Kind : int {
-    K_F1 = 0, K_F2, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B5, K_MISC,
+    K_F1 = 0, K_F2, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B34, K_B5, K_MISC,
     K_L_FWD, K_L_DB, K_L_DW, K_L_DX, K_RECOMP, K_CTR, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "B1.db_colsum",
     "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
-    "B5.dgrad_dX_shard_sum", "misc",
+    "B3+B4.wgrad_dB_dA",     "B5.dgrad_dX_shard_sum", "misc",
     "L.fwd_gemm_bias",       "L.dbias_colsum",        "L.wgrad_dW",      "L.dgrad_dX",
     "R.recompute_activation", "S.counter_reset",
 };
@@ -285,6 +285,10 @@ int resolve_sched(GemmArgs& g, const SchedReq& req, int64_t P, bool splittable) 
     g.sched = SCHED_TILES;
     g.groups = 1;
     g.kb_per_group = g.k_blocks;
+    if (g.second) {  // a grouped launch: whole tiles of both products
+        const int64_t all = tiles + static_cast<int64_t>(g.num_m_blocks2) * g.num_n_blocks2;
+        return static_cast<int>(std::min(all, P));
+    }
     const bool have_ws = g.partials != nullptr && g.counters != nullptr && splittable &&
                          g.colsum_out == nullptr;
     if (req.kind == SCHED_GROUPS && have_ws && req.groups > 1 && g.k_blocks % req.groups == 0) {
@@ -338,10 +342,20 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
     return launch_dep(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1, g);
 }
 
+// A second product launched with the first (grouped launch, whole tiles):
+// Aop2 · Bop2 into the M2 × N2 fp32 matrix out2, same K and layouts.
+struct SecondProduct {
+    const void* A;
+    const void* B;
+    int M, N;
+    void* out;
+};
+
 // Same product on CTA pairs: 256 × BN tiles, grid = 2 × (co-resident pairs).
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int K,
-                             const SchedReq& req, GemmArgs g, cudaStream_t st) {
+                             const SchedReq& req, GemmArgs g, cudaStream_t st,
+                             const SecondProduct* second = nullptr) {
     using Cfg = Tile2Cfg<BN>;
     const DeviceInfo* dev = device_info();
     if (dev == nullptr) return TPMLP_ERR_CUDA;
@@ -350,6 +364,21 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     const bool okB = B_MN ? make_map(&tmB, Bop, K, N, 64) : make_map(&tmB, Bop, N, K, BN / 2);
     CUtensorMap tmO0, tmO1;
     if (!okA || !okB || !make_out_maps<EPI>(&tmO0, &tmO1, g, M, N)) return TPMLP_ERR_CUDA;
+    CUtensorMap tmA2 = tmA, tmB2 = tmB;
+    if (second != nullptr) {
+        // the second product's output takes the second output map
+        if constexpr (EpiTraits<EPI>::kAct) return TPMLP_ERR_INVALID;
+        const SecondProduct& q = *second;
+        const bool ok2 = (A_MN ? make_map(&tmA2, q.A, K, q.M, 64) : make_map(&tmA2, q.A, q.M, K, kBM)) &&
+                         (B_MN ? make_map(&tmB2, q.B, K, q.N, 64) : make_map(&tmB2, q.B, q.N, K, BN / 2)) &&
+                         make_out_map(&tmO1, q.out, q.M, q.N, EPI == EPI_F32);
+        if (!ok2) return TPMLP_ERR_CUDA;
+        g.second = 1;
+        g.M2 = q.M;
+        g.N2 = q.N;
+        g.num_m_blocks2 = (q.M + kPairM - 1) / kPairM;
+        g.num_n_blocks2 = (q.N + BN - 1) / BN;
+    }
     g.M = M;
     g.N = N;
     g.K = K;
@@ -391,7 +420,7 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     // never more workers than the plan sized the workspace for (num_sms / 2)
     const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2), kSplittable<EPI, RELAY>);
     return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
-                      g);
+                      tmA2, tmB2, g);
 }
 
 // Algorithmic bytes of one GEMM: both operands read once (bf16), the
@@ -436,6 +465,29 @@ tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, i
         if (k_per_unit < threshold)
             return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, req, g, st);
         return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, req, g, st);
+    });
+}
+
+// Two products of the same kernel (fp32 epilogue) and K in one launch, as
+// one list of whole tiles on the CTA pairs (both M > 128): the second's
+// tiles follow the first's, so a short product no longer leaves half the
+// GPU idle for its whole duration.
+template <int BN, bool A_MN, bool B_MN>
+tpmlp_status gemm_tc_grouped(int kind, const void* A0, const void* B0, int M0, int N0, void* out0,
+                             const void* A1, const void* B1, int M1, int N1, void* out1, int K,
+                             cudaStream_t st) {
+    const double flops = 2.0 * (double(M0) * N0 + double(M1) * N1) * K;
+    const double bytes = gemm_bytes<EPI_F32>(M0, N0, K) + gemm_bytes<EPI_F32>(M1, N1, K);
+    return timed(kind, flops, bytes, st, [&] {
+        GemmArgs g{};
+        g.out0 = out0;
+        g.ld_out = N0;
+        const SecondProduct second{A1, B1, M1, N1, out1};
+        if (K < kRelayMinKPlain)
+            return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, false>(A0, B0, M0, N0, K, SchedReq{}, g, st,
+                                                                 &second);
+        return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, true>(A0, B0, M0, N0, K, SchedReq{}, g, st,
+                                                            &second);
     });
 }
 
@@ -534,7 +586,9 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
     SplitSpace sp;
     if (pl->tc && T > 0) {
         const int sms = plan_num_sms();
-        pl->f1 = plan_sched(T, F, h, 0, sms, &sp);                   // X·A
+        // X·A: whole tiles when the GeLU epilogue relays (K = h ≥ 3072), whose
+        // kernel has no split path
+        pl->f1 = plan_sched(T, F, h, 0, sms, &sp, h < kRelayMinKAct);
         pl->f2 = plan_sched(T, h, F, shard_groups(F, p), sms, &sp);  // Σ Y_i·B_i
         // dZ·Bᵀ: whole tiles when its relaying epilogue also sums da's columns
         // (those sums pair the rows of two warps, which a split tile, finished
@@ -949,17 +1003,23 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
             TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f,
                              da, st));
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
-        GemmArgs g3{};
-        set_split_space(g3, workspace, pl.off_part, pl.off_ctr);
-        g3.out0 = dB;
-        g3.ld_out = h;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, pl.b3, g3, st)));
         // B4: dA = Xᵀ·dH. Aop = X [T][h] (MN-major, M = h), Bop = dH [T][F] (MN-major).
-        GemmArgs g4{};
-        set_split_space(g4, workspace, pl.off_part, pl.off_ctr);
-        g4.out0 = dA;
-        g4.ld_out = F;
-        TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, pl.b4, g4, st)));
+        // Same kernel and K = T: one launch of both when both run whole tiles.
+        if (pl.b3.kind == SCHED_TILES && pl.b4.kind == SCHED_TILES && F > kBM && h > kBM) {
+            TPMLP_TRY((gemm_tc_grouped<256, true, true>(K_B34, Y, dZ, iF, ih, dB, X, dH, ih, iF, dA,
+                                                        iT, st)));
+        } else {
+            GemmArgs g3{};
+            set_split_space(g3, workspace, pl.off_part, pl.off_ctr);
+            g3.out0 = dB;
+            g3.ld_out = h;
+            TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, pl.b3, g3, st)));
+            GemmArgs g4{};
+            set_split_space(g4, workspace, pl.off_part, pl.off_ctr);
+            g4.out0 = dA;
+            g4.ld_out = F;
+            TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, pl.b4, g4, st)));
+        }
         // B5: dX = Σ_i dH_i·A_iᵀ. Aop = dH [T][F] (K-major), Bop = A [h][F] (K-major).
         GemmArgs g5{};
         set_split_space(g5, workspace, pl.off_part, pl.off_ctr);
