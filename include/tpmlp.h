@@ -216,6 +216,18 @@ int tpmlp_get_split_policy(void);
 void tpmlp_set_launch_overlap(int on);
 int tpmlp_get_launch_overlap(void);
 
+/* Dynamic tile schedule (default on). The SMs of a GPU do not all run a tile
+ * in the same time (measured on B200: the slowest CTA pairs take ~5% longer,
+ * the same pairs in every product), so with a static round-robin of tiles a
+ * long product ends with its slowest pair. With this on, the tensor-core
+ * products that run at least 4 waves of tiles on CTA pairs hand their tiles
+ * (and their stream-K segments) out in order from a counter in the
+ * workspace: faster pairs take more. Which pair computes a tile does not
+ * change the arithmetic: results are bit-identical with it on or off.
+ * A call that uses it zeroes its counters with one small kernel first. */
+void tpmlp_set_dynamic_schedule(int on);
+int tpmlp_get_dynamic_schedule(void);
+
 /* Upper bound, in nanoseconds, on any single wait inside a kernel (for data
  * from the tensor-memory accelerator, for the tensor cores, between warps).
  * Default 2e9 (2 s). A wait that runs out sets the device status word to

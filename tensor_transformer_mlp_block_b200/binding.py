@@ -25,7 +25,8 @@ EXPORTS = (
     "tpmlp_linear_workspace_size", "tp_linear_fwd", "tp_linear_bwd",
     "tp_mlp_recompute_activation", "tp_mlp_recompute_hidden", "tpmlp_strerror",
     "tpmlp_last_device_status", "tpmlp_set_split_policy", "tpmlp_get_split_policy",
-    "tpmlp_set_launch_overlap", "tpmlp_get_launch_overlap",
+    "tpmlp_set_launch_overlap", "tpmlp_get_launch_overlap", "tpmlp_set_dynamic_schedule",
+    "tpmlp_get_dynamic_schedule",
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
     "tpmlp_profile_read", "tpmlp_profile_reset", "tp_mlp_bwd_noalloc",
@@ -94,6 +95,9 @@ def lib() -> ctypes.CDLL:
             L.tpmlp_set_launch_overlap.argtypes = [ctypes.c_int]
             L.tpmlp_set_launch_overlap.restype = None
             L.tpmlp_get_launch_overlap.restype = ctypes.c_int
+            L.tpmlp_set_dynamic_schedule.argtypes = [ctypes.c_int]
+            L.tpmlp_set_dynamic_schedule.restype = None
+            L.tpmlp_get_dynamic_schedule.restype = ctypes.c_int
             L.tpmlp_set_wait_limit_ns.argtypes = [ctypes.c_uint64]
             L.tpmlp_set_wait_limit_ns.restype = None
             L.tpmlp_wait_selftest.argtypes = [ctypes.c_uint64, vp]
@@ -255,6 +259,14 @@ def set_split_policy(policy: int) -> None:
 
 def get_split_policy() -> int:
     return int(lib().tpmlp_get_split_policy())
+
+
+def set_dynamic_schedule(on: bool) -> None:
+    lib().tpmlp_set_dynamic_schedule(1 if on else 0)
+
+
+def get_dynamic_schedule() -> bool:
+    return bool(lib().tpmlp_get_dynamic_schedule())
 
 
 def set_launch_overlap(on: bool) -> None:

@@ -97,6 +97,12 @@ struct GemmArgs {
     // M2 × N2 tiles follow the first product's. second = 0: none.
     int second;
     int M2, N2, num_m_blocks2, num_n_blocks2;
+    // Dynamic schedule (CTA-pair kernel; null: static round-robin). Work
+    // items are taken in order from dyn_counter[0] by each pair's leader
+    // producer and handed to the pair's other roles through a shared-memory
+    // queue; the last pair to finish puts dyn_counter[0..1] back to zero.
+    // Both must be zero at launch.
+    int* dyn_counter;
 };
 
 constexpr int kBM = 128;
@@ -248,6 +254,209 @@ TPMLP_HD bool next_unit(const GemmArgs& g, WorkIter& it, WorkUnit& w) {
     w.key = st;
     it.cur += w.kb1 - w.kb0;
     return true;
+}
+
+// ------------------------------------------------- dynamic schedule (pairs)
+// A tile costs the same on every SM, but the SMs do not run at the same
+// speed (measured: the slowest CTA pairs take ~5% longer per tile, the same
+// pairs in every product). With a static round-robin the product ends with
+// its slowest pair; with items taken in order from a global counter, fast
+// pairs take more of them. Items are the schedule's units (whole tiles, shard
+// group units) or, for the stream-K tail, whole tiles and then one item per
+// segment, which expands into the segment's pieces in every role the same
+// way. Results do not depend on which pair runs an item.
+
+constexpr int kQueue = 8;  // item slots of a pair's queue
+
+TPMLP_HD int dyn_items(const GemmArgs& g, int P) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    if (g.sched == SCHED_GROUPS) return tiles * g.groups;
+    if (g.sched == SCHED_STREAMK) return sk_whole_tiles(g, P) + (sk_work(g, P) > 0 ? P : 0);
+    return tiles + (g.second ? g.num_m_blocks2 * g.num_n_blocks2 : 0);
+}
+
+// The first unit of item `id`. For a stream-K segment, `it` yields its other
+// pieces afterwards (seg = true); any other item is a single unit.
+TPMLP_HD bool dyn_item_first(const GemmArgs& g, int P, int id, WorkIter& it, bool& seg, WorkUnit& w) {
+    seg = false;
+    if (g.sched == SCHED_STREAMK && id >= sk_whole_tiles(g, P)) {
+        const int j = id - sk_whole_tiles(g, P);  // the segment, as the static schedule's worker j
+        it = work_iter(j, P);
+        it.tail = true;
+        const int64_t W = sk_work(g, P);
+        it.cur = sk_begin(j, W, P);
+        it.end = sk_begin(j + 1, W, P);
+        seg = true;
+        return next_unit(g, it, w);
+    }
+    it = work_iter(id, P);  // the static schedule's unit number `id`
+    return next_unit(g, it, w);
+}
+
+// This CTA's view of its pair's item queue.
+struct PairQueue {
+    uint32_t items;  // shared address of kQueue item ids (this CTA's copy)
+    uint32_t full;   // kQueue barriers of this CTA: slot s holds an item
+    uint32_t empty;  // kQueue barriers of the leader: every role has read slot s
+    bool leader;     // this CTA is the pair's leader
+};
+
+// A consumer role (the leader's MMA thread and epilogue warps, the other
+// CTA's producer and epilogue warps) takes the id in slot n mod kQueue.
+// WARP: all lanes wait and read; lane 0 arrives. False: a wait gave up.
+template <bool WARP>
+__device__ __forceinline__ bool queue_take(const PairQueue& q, int n, int& id, volatile int* abort,
+                                           uint64_t limit) {
+    const int s = n % kQueue;
+    const uint32_t par = static_cast<uint32_t>(n / kQueue) & 1u;
+    // the other CTA's copy arrives with a release at cluster scope
+    bool got = mbar_wait_bounded_cluster(q.full + 8 * s, par, abort, limit);
+    if (WARP) got = __all_sync(0xffffffffu, got);
+    if (!got) return false;
+    id = static_cast<int>(ld_shared_u32(q.items + 4 * s));
+    if (!WARP || (threadIdx.x & 31) == 0) {
+        const uint32_t e = q.empty + 8 * s;
+        if (q.leader)
+            mbar_arrive(e);
+        else
+            mbar_arrive_cluster(mapa_shared(e, 0));
+    }
+    if (WARP) __syncwarp();
+    return true;
+}
+
+// The leader's producer puts item `id` (-1: past the end) into slot
+// n mod kQueue of both CTAs' queues, once every role has read the slot's
+// previous item.
+__device__ __forceinline__ bool queue_publish(const PairQueue& q, int n, int id, volatile int* abort,
+                                              uint64_t limit) {
+    const int s = n % kQueue;
+    const uint32_t par = static_cast<uint32_t>(n / kQueue) & 1u;
+    if (!mbar_wait_bounded_cluster(q.empty + 8 * s, par ^ 1u, abort, limit)) return false;
+    const uint32_t slot = q.items + 4 * s;
+    asm volatile("st.volatile.shared.u32 [%0], %1;" ::"r"(slot), "r"(id) : "memory");
+    st_shared_cluster_u32(mapa_shared(slot, 1), static_cast<uint32_t>(id));
+    mbar_arrive(q.full + 8 * s);
+    mbar_arrive_cluster(mapa_shared(q.full + 8 * s, 1));
+    return true;
+}
+
+// Where a role's units come from: the static sequence of its worker, or
+// the items of the pair's queue (dynamic schedule).
+struct UnitCursor {
+    WorkIter it;   // static: the worker's sequence; dynamic: the current segment's pieces
+    bool dyn;
+    bool seg;      // dynamic: `it` may have pieces of the current item left
+    int n;         // dynamic: items taken (consumers) or published (leader's producer)
+    // leader's producer: the item published one ahead of the one it loads,
+    // and the counter value drawn for the item after that (still in flight)
+    int ahead, pend;
+    bool started;
+};
+
+__device__ __forceinline__ UnitCursor unit_cursor(int worker, int nworkers, bool dyn) {
+    UnitCursor c;
+    c.it = work_iter(worker, nworkers);
+    c.dyn = dyn;
+    c.seg = false;
+    c.n = 0;
+    c.ahead = -1;
+    c.pend = -1;
+    c.started = false;
+    return c;
+}
+
+// The leader's producer: the next item to load. Items are published one
+// ahead of the one being loaded, and the counter draw for the item after
+// that is issued right away and used one item later, so the atomic's latency
+// hides behind the current item's loads (a tile's loads never wait for it).
+__device__ __forceinline__ bool give_next_item(const GemmArgs& g, int items, UnitCursor& c, int& id,
+                                               const PairQueue& q, volatile int* abort,
+                                               uint64_t limit) {
+    if (!c.started) {
+        c.started = true;
+        int first = atomicAdd(g.dyn_counter, 1);
+        if (first >= items) first = -1;
+        if (!queue_publish(q, c.n++, first, abort, limit)) return false;
+        c.ahead = first;
+        c.pend = first >= 0 ? atomicAdd(g.dyn_counter, 1) : -1;
+    }
+    id = c.ahead;
+    if (id < 0) return true;
+    int next = c.pend;
+    if (next >= items) next = -1;
+    if (!queue_publish(q, c.n++, next, abort, limit)) return false;
+    c.ahead = next;
+    c.pend = next >= 0 ? atomicAdd(g.dyn_counter, 1) : -1;
+    return true;
+}
+
+// The whole tile numbered u of a whole-tile schedule (the second product's
+// tiles follow the first's).
+__device__ __forceinline__ void whole_tile_unit(const GemmArgs& g, int u, WorkUnit& w) {
+    const int tiles = g.num_m_blocks * g.num_n_blocks;
+    w.prob = u < tiles ? 0 : 1;
+    if (w.prob == 0)
+        tile_coords(g, u, w.mb, w.nb);
+    else
+        tile_coords_of(g.num_m_blocks2, g.num_n_blocks2, u - tiles, w.mb, w.nb);
+    w.kb0 = 0;
+    w.kb1 = g.k_blocks;
+    w.pieces = 1;
+    w.piece = 0;
+    w.key = 0;
+    w.seg_lo = 0;
+}
+
+// The next unit of a role; false at the end, or (ok = false) when a wait gave
+// up. GIVE: the leader's producer, which draws the items. TILES_ONLY: the
+// kernel runs whole-tile schedules only (fewer registers live).
+template <bool GIVE, bool WARP, bool TILES_ONLY = false>
+__device__ __forceinline__ bool cursor_next(const GemmArgs& g, int P, UnitCursor& c, WorkUnit& w,
+                                            const PairQueue* q, bool& ok, volatile int* abort,
+                                            uint64_t limit) {
+    if constexpr (TILES_ONLY) {
+        int u;
+        if (!c.dyn) {
+            u = c.it.worker + c.it.next * c.it.nworkers;
+            ++c.it.next;
+            const int all = g.num_m_blocks * g.num_n_blocks +
+                            (g.second ? g.num_m_blocks2 * g.num_n_blocks2 : 0);
+            if (u >= all) return false;
+        } else {
+            const bool got = GIVE ? give_next_item(g, dyn_items(g, P), c, u, *q, abort, limit)
+                                  : queue_take<WARP>(*q, c.n, u, abort, limit);
+            if (!got) {
+                ok = false;
+                return false;
+            }
+            if (!GIVE) ++c.n;
+            if (u < 0) return false;
+        }
+        whole_tile_unit(g, u, w);
+        return true;
+    }
+    if (!c.dyn) return next_unit(g, c.it, w);
+    for (;;) {
+        if (c.seg) {
+            if (next_unit(g, c.it, w)) return true;
+            c.seg = false;
+        }
+        int id = -1;
+        const bool got = GIVE ? give_next_item(g, dyn_items(g, P), c, id, *q, abort, limit)
+                              : queue_take<WARP>(*q, c.n, id, abort, limit);
+        if (!got) {
+            ok = false;
+            return false;
+        }
+        if (!GIVE) ++c.n;
+        if (id < 0) return false;
+        bool seg = false;
+        if (dyn_item_first(g, P, id, c.it, seg, w)) {
+            c.seg = seg;
+            return true;
+        }
+    }
 }
 
 // Workspace slot (one partial tile) of piece q of a split tile. Shard groups:
@@ -674,7 +883,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                                               uint64_t* xempty, uint8_t* sEpi, int worker,
                                               int nworkers, int tile_rows, int cta_row_off,
                                               volatile int* abort, uint64_t limit, int warp,
-                                              int lane) {
+                                              int lane, const PairQueue* queue = nullptr) {
     constexpr int kChunks = BN / 64;  // 32-column chunks per half of the tile
     const int quad = warp & 3;          // tensor-memory lanes this warp may access
     const int half = (warp - 2) / 4;    // which half of the tile's columns
@@ -690,9 +899,12 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     }
     uint32_t xcount = 0;
     bool stored = false;  // a relay warp has bulk stores of a split tile in flight
-    WorkIter it = work_iter(worker, nworkers);
+    UnitCursor cur = unit_cursor(worker, nworkers, queue != nullptr);
     WorkUnit w;
-    for (int local = 0; next_unit(g, it, w); ++local) {
+    bool qok = true;
+    for (int local = 0;
+         cursor_next<false, true, !kSplittable<EPI, RELAY>>(g, nworkers, cur, w, queue, qok, abort, limit);
+         ++local) {
         const int buf = local & 1;
         const uint32_t aphase = (local >> 1) & 1;
         // every lane waits; the warp proceeds only if all lanes saw the
@@ -853,6 +1065,7 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
             break;
         }
     }
+    if (!qok) raise_timeout(abort);
     if (lane == 0) bulk_wait0();  // this warp's stores are complete before exit
     __syncwarp();
 }

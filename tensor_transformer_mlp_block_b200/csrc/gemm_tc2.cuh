@@ -30,7 +30,9 @@ struct Tile2Cfg {
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
     static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
     static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
-    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5 + 8) + 16;
+    // barriers: ring (2·STAGES), accumulators (4), drain, relay (8), item
+    // queue (2·kQueue); then the TMEM address, the abort flag, the queue's items
+    static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5 + 8 + 2 * kQueue) + 16 + 4 * kQueue;
     static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
 };
 
@@ -60,8 +62,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint64_t* drain = bars + 2 * STAGES + 4;
     uint64_t* xfull = bars + 2 * STAGES + 5;   // relay hand-off, 4 pairs
     uint64_t* xempty = bars + 2 * STAGES + 9;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 2 * STAGES + 13);
+    uint64_t* qfull = bars + 2 * STAGES + 13;  // item queue (dynamic schedule)
+    uint64_t* qempty = qfull + kQueue;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(qempty + kQueue);
     volatile int* abort = reinterpret_cast<volatile int*>(tmem_slot + 1);
+    int* qitems = reinterpret_cast<int*>(tmem_slot + 4);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -84,6 +89,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&xfull[x]), 32);
             mbar_init(smem_u32(&xempty[x]), 32);
         }
+        // readers of each queue slot: the leader's MMA thread and 8 epilogue
+        // warps, the other CTA's producer and 8 epilogue warps
+        for (int x = 0; x < kQueue; ++x) {
+            mbar_init(smem_u32(&qfull[x]), 1);
+            mbar_init(smem_u32(&qempty[x]), 2 + 2 * kEpiWarps);
+        }
         *abort = 0;
         fence_mbar_init();
     }
@@ -102,6 +113,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const uint64_t limit = g.wait_limit_ns;  // num_m_blocks counts 256-row blocks
     if (warp == 0) zero_later_counters(g, lane);
+    const bool dyn = g.dyn_counter != nullptr;
+    const PairQueue queue{smem_u32(qitems), smem_u32(qfull), smem_u32(qempty), leader};
 
     if (warp == 0) {
         // ------------------------------------------------ TMA producer (both CTAs)
@@ -118,9 +131,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             bool ok = true;
             const int a_row0 = static_cast<int>(rank) * kBM;
             const int b_col0 = static_cast<int>(rank) * (BN / 2);
-            WorkIter it = work_iter(pair, npairs);
+            UnitCursor cur = unit_cursor(pair, npairs, dyn);
             WorkUnit w;
-            while (ok && next_unit(g, it, w)) {
+            bool qok = true;
+            while (ok && (leader ? cursor_next<true, false>(g, npairs, cur, w, &queue, qok, abort, limit)
+                                 : cursor_next<false, false>(g, npairs, cur, w, &queue, qok, abort, limit))) {
                 const int mb = w.mb, nb = w.nb;
                 const int kb0 = w.kb0, kb1 = w.kb1;
                 const CUtensorMap* mA = w.prob ? &tmA2 : &tmA;
@@ -156,6 +171,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                         stage = 0;
                         phase ^= 1u;
                     }
+                }
+            }
+            if (!qok) {
+                raise_timeout(abort);
+                ok = false;
+            }
+            if (dyn && leader && ok) {
+                // every pair has drawn past the end once it arrives here: the
+                // last one puts the counters back to zero for the next launch
+                __threadfence();
+                if (atomicAdd(g.dyn_counter + 1, 1) == npairs - 1) {
+                    atomicExch(g.dyn_counter, 0);
+                    atomicExch(g.dyn_counter + 1, 0);
                 }
             }
             if (ok && !*abort) {
@@ -195,9 +223,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            WorkIter it = work_iter(pair, npairs);
+            UnitCursor cur = unit_cursor(pair, npairs, dyn);
             WorkUnit w;
-            for (int local = 0; ok && next_unit(g, it, w); ++local) {
+            bool qok = true;
+            for (int local = 0;
+                 ok && cursor_next<false, false>(g, npairs, cur, w, &queue, qok, abort, limit); ++local) {
                 const int kb0 = w.kb0, kb1 = w.kb1;
                 const int buf = local & 1;
                 const uint32_t aphase = (local >> 1) & 1;
@@ -234,6 +264,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                 if (!ok) break;
                 umma_commit_pair(smem_u32(&tfull[buf]), 0x3);
             }
+            if (!qok) {
+                raise_timeout(abort);
+                ok = false;
+            }
             if (!ok || *abort) {
                 umma_commit_pair(smem_u32(drain), 0x1);
                 volatile int never = 0;
@@ -245,7 +279,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         // ------------------------------------------------ epilogue warps (both CTAs)
         epilogue_role<BN, EPI, true, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
                                             pair, npairs, kPairM, static_cast<int>(rank) * kBM, abort,
-                                            limit, warp, lane);
+                                            limit, warp, lane, dyn ? &queue : nullptr);
     }
 
     tc_fence_before();

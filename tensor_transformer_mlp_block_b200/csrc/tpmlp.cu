@@ -43,6 +43,7 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_split_policy{0};
 std::atomic<bool> g_overlap{true};  // programmatic dependent launches
+std::atomic<bool> g_dynamic{true};  // dynamic tile schedule for long products
 
 struct DeviceInfo {
     bool init = false;
@@ -250,6 +251,7 @@ struct SchedReq {
     int kind = SCHED_TILES;  // SCHED_TILES, SCHED_GROUPS or SCHED_STREAMK
     int groups = 1;          // SCHED_GROUPS: consecutive k ranges per tile
     bool force = false;      // SCHED_STREAMK even where the time model says it does not pay
+    bool dyn = false;        // items handed out dynamically (CTA pairs; needs the counters)
 };
 
 // Shortest stream-K segment allowed, and the tail's extra cost (partial
@@ -339,6 +341,7 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
         }
     }
     const int grid = resolve_sched(g, req, dev->num_sms, kSplittable<EPI, RELAY>);
+    g.dyn_counter = nullptr;  // the one-CTA kernel runs the static schedule
     return launch_dep(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1, g);
 }
 
@@ -419,6 +422,7 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     }
     // never more workers than the plan sized the workspace for (num_sms / 2)
     const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2), kSplittable<EPI, RELAY>);
+    if (!req.dyn) g.dyn_counter = nullptr;
     return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
                       tmA2, tmB2, g);
 }
@@ -475,18 +479,21 @@ tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, i
 template <int BN, bool A_MN, bool B_MN>
 tpmlp_status gemm_tc_grouped(int kind, const void* A0, const void* B0, int M0, int N0, void* out0,
                              const void* A1, const void* B1, int M1, int N1, void* out1, int K,
-                             cudaStream_t st) {
+                             int* dyn_counter, cudaStream_t st) {
     const double flops = 2.0 * (double(M0) * N0 + double(M1) * N1) * K;
     const double bytes = gemm_bytes<EPI_F32>(M0, N0, K) + gemm_bytes<EPI_F32>(M1, N1, K);
     return timed(kind, flops, bytes, st, [&] {
         GemmArgs g{};
         g.out0 = out0;
         g.ld_out = N0;
+        g.dyn_counter = dyn_counter;
+        SchedReq req;
+        req.dyn = dyn_counter != nullptr;
         const SecondProduct second{A1, B1, M1, N1, out1};
         if (K < kRelayMinKPlain)
-            return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, false>(A0, B0, M0, N0, K, SchedReq{}, g, st,
+            return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, false>(A0, B0, M0, N0, K, req, g, st,
                                                                  &second);
-        return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, true>(A0, B0, M0, N0, K, SchedReq{}, g, st,
+        return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, true>(A0, B0, M0, N0, K, req, g, st,
                                                             &second);
     });
 }
@@ -522,6 +529,22 @@ struct SplitSpace {
         counter_bytes = std::max(counter_bytes, ctr);
     }
 };
+
+// Two ints after the split counters: the dynamic schedule's item counter and
+// its count of finished pairs (zero at every launch; the last pair resets them).
+constexpr size_t kDynCounterInts = 2;
+
+// Whether a product runs the dynamic schedule: on CTA pairs (M > 128), with
+// at least 4 waves of items and at least 192 k-blocks per tile. Measured on
+// B200 (same run, alternating): 1.5–2% faster for the 175B-class products
+// with 192–768 k-blocks per tile; no gain with 64–256 (7B-class), and 6%
+// slower with 32 (the 175B-class weight gradients: each item's hand-off
+// costs a fixed time that a short tile does not amortise).
+bool wants_dynamic(int64_t M, int64_t items, int64_t K, int num_sms) {
+    return g_dynamic.load() && M > kBM && items >= 4 * (num_sms / 2) && (K + kBK - 1) / kBK >= 192;
+}
+
+int64_t pair_tiles(int64_t M, int64_t N) { return ((M + kPairM - 1) / kPairM) * ((N + 255) / 256); }
 
 // Schedule of one tensor-core product (M × N output, K deep) under the
 // current policy (tpmlp_set_split_policy):
@@ -575,8 +598,10 @@ struct Plan {
     bool tc = false;    // tensor-core path (bf16, h % 8 == 0, F % 8 == 0)
     SchedReq f1, f2, b2, b3, b4, b5;
     bool fwd_split = false, bwd_split = false;  // some product of the call splits tiles
+    bool fwd_dyn = false, bwd_dyn = false;      // some product of the call is dynamic
+    bool group34 = false;                       // B3 and B4 in one launch
     int64_t chunks = 1; // column-sum row chunks
-    size_t off_part = 0, off_ctr = 0, ctr_bytes = 0, off_cs_h = 0, off_cs_f = 0, total = 0;
+    size_t off_part = 0, off_ctr = 0, off_dyn = 0, ctr_bytes = 0, off_cs_h = 0, off_cs_f = 0, total = 0;
 };
 
 bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl) {
@@ -600,13 +625,34 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
         pl->fwd_split = pl->f1.kind != SCHED_TILES || pl->f2.kind != SCHED_TILES;
         pl->bwd_split = pl->b2.kind != SCHED_TILES || pl->b3.kind != SCHED_TILES ||
                         pl->b4.kind != SCHED_TILES || pl->b5.kind != SCHED_TILES;
+        pl->group34 = pl->b3.kind == SCHED_TILES && pl->b4.kind == SCHED_TILES && F > kBM && h > kBM;
+        // items of each product (a split tile's units count as items too)
+        auto items = [&](const SchedReq& r, int64_t M, int64_t N) {
+            return pair_tiles(M, N) * (r.kind == SCHED_GROUPS ? r.groups : 1);
+        };
+        pl->f1.dyn = wants_dynamic(T, items(pl->f1, T, F), h, sms);
+        pl->f2.dyn = wants_dynamic(T, items(pl->f2, T, h), F, sms);
+        pl->b2.dyn = wants_dynamic(T, items(pl->b2, T, F), h, sms);
+        if (pl->group34) {
+            pl->b3.dyn = pl->b4.dyn =
+                wants_dynamic(std::min(F, h), pair_tiles(F, h) + pair_tiles(h, F), T, sms);
+        } else {
+            pl->b3.dyn = wants_dynamic(F, items(pl->b3, F, h), T, sms);
+            pl->b4.dyn = wants_dynamic(h, items(pl->b4, h, F), T, sms);
+        }
+        pl->b5.dyn = wants_dynamic(T, items(pl->b5, T, h), F, sms);
+        pl->fwd_dyn = pl->f1.dyn || pl->f2.dyn;
+        pl->bwd_dyn = pl->b2.dyn || pl->b3.dyn || pl->b4.dyn || pl->b5.dyn;
     }
     pl->chunks = T > 0 ? (T + kColsumRowsPerChunk - 1) / kColsumRowsPerChunk : 1;
     size_t off = 0;
     pl->off_part = off;
     off += round256(sp.partial_bytes);
     pl->off_ctr = off;
-    pl->ctr_bytes = round256(sp.counter_bytes);
+    pl->off_dyn = pl->off_ctr + sp.counter_bytes;  // the dynamic schedule's two ints
+    pl->ctr_bytes = (pl->fwd_dyn || pl->bwd_dyn)
+                        ? round256(sp.counter_bytes + kDynCounterInts * sizeof(int))
+                        : round256(sp.counter_bytes);
     off += pl->ctr_bytes;
     pl->off_cs_h = off;
     off += round256(static_cast<size_t>(pl->chunks) * h * sizeof(float));
@@ -710,6 +756,11 @@ tpmlp_status reset_counters(void* workspace, size_t off, size_t bytes, cudaStrea
 void set_split_space(GemmArgs& g, void* workspace, size_t off_part, size_t off_ctr) {
     g.partials = reinterpret_cast<float*>(static_cast<char*>(workspace) + off_part);
     g.counters = reinterpret_cast<int*>(static_cast<char*>(workspace) + off_ctr);
+}
+
+// The dynamic schedule's counters (used only by a launch whose request says so).
+int* dyn_space(void* workspace, size_t off_dyn) {
+    return reinterpret_cast<int*>(static_cast<char*>(workspace) + off_dyn);
 }
 
 // The counters must be zero before the first product of a call that splits
@@ -909,8 +960,13 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
         const SchedReq f1 = with_f2 ? pl.f1 : SchedReq{};
         // F1: H = X·A + a, Y = GeLU(H). Aop = X [T][h] (K-major), Bop = A [h][F] (MN-major).
         GemmArgs g1{};
-        if (with_f2) set_split_space(g1, workspace, pl.off_part, pl.off_ctr);
-        if (with_f2 && pl.fwd_split)
+        if (with_f2) {
+            set_split_space(g1, workspace, pl.off_part, pl.off_ctr);
+            g1.dyn_counter = dyn_space(workspace, pl.off_dyn);
+        }
+        if (with_f2 && pl.fwd_dyn)  // the first product itself needs them zero
+            TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
+        else if (with_f2 && pl.fwd_split)
             TPMLP_TRY(zero_counters_before(g1, f1, workspace, pl.off_ctr, pl.ctr_bytes, st));
         g1.out0 = H;
         g1.out1 = Y;
@@ -924,6 +980,7 @@ tpmlp_status fwd_impl(const void* X, const void* A, const void* a, const void* B
         // order in the epilogue of the last one, then b once.
         GemmArgs g2{};
         set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
+        g2.dyn_counter = dyn_space(workspace, pl.off_dyn);
         g2.out0 = Z;
         g2.ld_out = h;
         g2.bias = static_cast<const __nv_bfloat16*>(b);
@@ -980,6 +1037,8 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
             if (!aligned16(q)) return TPMLP_ERR_ALIGN;
         const int iT = static_cast<int>(T), ih = static_cast<int>(h), iF = static_cast<int>(F);
         const __nv_bfloat16* dZb = static_cast<const __nv_bfloat16*>(dZ);
+        int* dyn = dyn_space(workspace, pl.off_dyn);
+        if (pl.bwd_dyn) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
         // db = 1ᵀ·dZ
         TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
@@ -990,7 +1049,9 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         const bool fused_da = h >= kRelayMinKAct;
         GemmArgs g2{};
         set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
-        if (pl.bwd_split) TPMLP_TRY(zero_counters_before(g2, pl.b2, workspace, pl.off_ctr, pl.ctr_bytes, st));
+        g2.dyn_counter = dyn;
+        if (pl.bwd_split && !pl.bwd_dyn)
+            TPMLP_TRY(zero_counters_before(g2, pl.b2, workspace, pl.off_ctr, pl.ctr_bytes, st));
         g2.out0 = dH;
         g2.ld_out = F;
         g2.aux = static_cast<const __nv_bfloat16*>(H);
@@ -1005,17 +1066,19 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
         // B4: dA = Xᵀ·dH. Aop = X [T][h] (MN-major, M = h), Bop = dH [T][F] (MN-major).
         // Same kernel and K = T: one launch of both when both run whole tiles.
-        if (pl.b3.kind == SCHED_TILES && pl.b4.kind == SCHED_TILES && F > kBM && h > kBM) {
+        if (pl.group34) {
             TPMLP_TRY((gemm_tc_grouped<256, true, true>(K_B34, Y, dZ, iF, ih, dB, X, dH, ih, iF, dA,
-                                                        iT, st)));
+                                                        iT, pl.b3.dyn ? dyn : nullptr, st)));
         } else {
             GemmArgs g3{};
             set_split_space(g3, workspace, pl.off_part, pl.off_ctr);
+            g3.dyn_counter = dyn;
             g3.out0 = dB;
             g3.ld_out = h;
             TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, pl.b3, g3, st)));
             GemmArgs g4{};
             set_split_space(g4, workspace, pl.off_part, pl.off_ctr);
+            g4.dyn_counter = dyn;
             g4.out0 = dA;
             g4.ld_out = F;
             TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, pl.b4, g4, st)));
@@ -1023,6 +1086,7 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // B5: dX = Σ_i dH_i·A_iᵀ. Aop = dH [T][F] (K-major), Bop = A [h][F] (K-major).
         GemmArgs g5{};
         set_split_space(g5, workspace, pl.off_part, pl.off_ctr);
+        g5.dyn_counter = dyn;
         g5.out0 = dX;
         g5.ld_out = h;
         TPMLP_TRY((gemm_tc<256, false, false, EPI_BIAS>(K_B5, dH, A, iT, ih, iF, pl.b5, g5, st)));
@@ -1229,6 +1293,10 @@ tpmlp_status tpmlp_set_split_policy(int policy) {
 int tpmlp_get_split_policy(void) { return g_split_policy.load(); }
 
 void tpmlp_set_launch_overlap(int on) { g_overlap.store(on != 0); }
+
+void tpmlp_set_dynamic_schedule(int on) { g_dynamic.store(on != 0); }
+
+int tpmlp_get_dynamic_schedule(void) { return g_dynamic.load() ? 1 : 0; }
 
 int tpmlp_get_launch_overlap(void) { return g_overlap.load() ? 1 : 0; }
 

@@ -119,6 +119,7 @@ def test_workspace_size_formula(lib):
     import torch
     from tensor_transformer_mlp_block_b200 import binding
     binding.set_split_policy(1)
+    binding.set_dynamic_schedule(False)
     try:
         for T, h, F, p in [(8192, 4096, 16384, 2), (300, 200, 520, 2), (1, 8, 8, 1), (129, 64, 264, 3)]:
             assert binding.workspace_size(T, h, F, p) == _colsums(T, h, F), (T, h, F)
@@ -143,8 +144,15 @@ def test_workspace_size_formula(lib):
         assert binding.plan_schedules(T, h, F, p)["F1"] == binding.SCHED_STREAMK
         assert binding.workspace_size(T, h, F, p) == (_r256(2 * 74 * 256 * 256 * 4)
                                                       + _r256(74 * 16 * 4) + _colsums(T, h, F))
+        # the dynamic schedule (products of ≥ 4 waves on CTA pairs) adds its two
+        # int counters after the split counters
+        binding.set_split_policy(1)
+        binding.set_dynamic_schedule(True)
+        assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20 + 256
+        assert binding.workspace_size(4096, 768, 3072, 2) == _colsums(4096, 768, 3072)  # < 4 waves
     finally:
         binding.set_split_policy(0)
+        binding.set_dynamic_schedule(True)
 
 
 def test_automatic_schedules_for_the_named_workloads(lib):
