@@ -216,15 +216,19 @@ int tpmlp_get_split_policy(void);
 void tpmlp_set_launch_overlap(int on);
 int tpmlp_get_launch_overlap(void);
 
-/* Dynamic tile schedule (default on). The SMs of a GPU do not all run a tile
- * in the same time (measured on B200: the slowest CTA pairs take ~5% longer,
- * the same pairs in every product), so with a static round-robin of tiles a
- * long product ends with its slowest pair. With this on, the tensor-core
- * products that run at least 4 waves of tiles on CTA pairs hand their tiles
- * (and their stream-K segments) out in order from a counter in the
+/* Dynamic tile schedule (default off). The SMs of a GPU do not all run a
+ * tile in the same time (measured on B200: the slowest CTA pairs take ~5%
+ * longer, the same pairs in every product), so with a static round-robin of
+ * tiles a long product ends with its slowest pair. With this on, the
+ * tensor-core products with bf16 outputs that run at least 4 waves of tiles
+ * on CTA pairs and at least 192 k-blocks (12288 of K) per tile hand their
+ * tiles (and their stream-K segments) out in order from a counter in the
  * workspace: faster pairs take more. Which pair computes a tile does not
  * change the arithmetic: results are bit-identical with it on or off.
- * A call that uses it zeroes its counters with one small kernel first. */
+ * A call that uses it zeroes its counters with one small kernel first.
+ * Off by default: a launch alone runs 2–3% faster with it, but a full
+ * forward + backward step, which runs at the GPU's power limit, did not get
+ * faster (measured on B200, alternating runs). */
 void tpmlp_set_dynamic_schedule(int on);
 int tpmlp_get_dynamic_schedule(void);
 

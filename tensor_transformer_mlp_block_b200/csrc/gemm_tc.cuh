@@ -748,19 +748,29 @@ __device__ __forceinline__ void unpack_bf16x8(const uint4& v, float* f) {
 // stores the whole chunk with a TMA bulk tensor store, which clips rows and
 // columns outside the output. The slot is reused only after the previous
 // store of this warp has finished reading it.
-template <int EPI>
+// DBL: the warp stages chunks alternately in two slots (slot_base and the
+// 4 KB after it), so a chunk's bulk store may still be reading one slot while
+// the next chunk is staged in the other; sbuf is the warp's toggle. It flips
+// only when a store group is committed (a chunk wholly outside the output
+// stores nothing), so the most recent group always read the other slot and
+// waiting for all but one group frees this one.
 // cs_mode (GeLU′ epilogues with colsum_out): 0 = none; 1 = keep this chunk's
 // stored values in csx; 2 = add them to csx, reduce csx over the 32 lanes
 // and write the column sums to colsum_out row cs_row (if cs_row ≥ 0).
+template <int EPI, bool DBL>
 __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensorMap* tmO0,
                                                const CUtensorMap* tmO1, const uint32_t (&acc)[32],
-                                               int row0, int col0, int M, int N, uint32_t slot,
-                                               int lane, float (&csx)[32], int cs_mode,
-                                               int64_t cs_row) {
+                                               int row0, int col0, int M, int N, uint32_t slot_base,
+                                               uint32_t& sbuf, int lane, float (&csx)[32],
+                                               int cs_mode, int64_t cs_row) {
+    const uint32_t slot = DBL ? slot_base + sbuf * kEpiSlotBytes : slot_base;
     const int row = row0 + lane;
     const bool any = (row0 < M) && (col0 < N);
     if constexpr (EPI == EPI_F32) {
-        if (lane == 0) bulk_wait_read0();
+        if (lane == 0) {
+            if (DBL) bulk_wait_read1();
+            else bulk_wait_read0();
+        }
         __syncwarp();
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
@@ -773,6 +783,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             tma_store_3d(tmO0, slot, col0, row0, 0);
             bulk_commit();
         }
+        if (DBL && any) sbuf ^= 1u;
     } else {
         uint4 o0[4], o1[4];
         const int64_t off = static_cast<int64_t>(row) * g.ld_out + col0;
@@ -815,7 +826,10 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
                 o1[q].w = pack_bf16x2(y[6], y[7]);
             }
         }
-        if (lane == 0) bulk_wait_read0();
+        if (lane == 0) {
+            if (DBL) bulk_wait_read1();
+            else bulk_wait_read0();
+        }
         __syncwarp();
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
@@ -830,6 +844,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
             if constexpr (EpiTraits<EPI>::kAct) tma_store_3d(tmO1, slot + 2048, col0, row0, 0);
             bulk_commit();
         }
+        if (DBL && any) sbuf ^= 1u;
         if constexpr (EpiTraits<EPI>::kDAct) {
             // da's partial from the values just stored (rows beyond M and
             // columns beyond N hold zeros): this lane's row of the chunk, then
@@ -876,7 +891,7 @@ __device__ __forceinline__ void epilogue_chunk(const GemmArgs& g, const CUtensor
 template <int EPI, bool RELAY>
 constexpr bool kSplittable = !((EpiTraits<EPI>::kDAct || EpiTraits<EPI>::kAct) && RELAY);
 
-template <int BN, int EPI, bool PAIR, bool RELAY>
+template <int BN, int EPI, bool PAIR, bool RELAY, bool DBL = false>
 __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorMap* tmO0,
                                               const CUtensorMap* tmO1, uint32_t tmem_base,
                                               uint64_t* tfull, uint64_t* tempty, uint64_t* xfull,
@@ -889,10 +904,12 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
     const int half = (warp - 2) / 4;    // which half of the tile's columns
     const bool relay = RELAY && quad < 2;
     const int pair_id = (quad & 1) + 2 * half;  // relay (quad 0/1) <-> math (quad 2/3)
-    const uint32_t slot = smem_u32(sEpi + (warp - 2) * kEpiSlotBytes);
+    constexpr int kSlotsPerWarp = DBL ? 2 : 1;
+    const uint32_t slot = smem_u32(sEpi + kSlotsPerWarp * (warp - 2) * kEpiSlotBytes);
+    uint32_t sbuf = 0;  // DBL: which of the warp's two slots stages the next chunk
     // a math warp's (quad 2/3) partner relay is warp 2 + 4·half + quad (quad - 2,
     // same half), whose slot index is 4·half + quad
-    const uint32_t partner_slot = smem_u32(sEpi + (4 * half + quad) * kEpiSlotBytes);
+    const uint32_t partner_slot = smem_u32(sEpi + kSlotsPerWarp * (4 * half + quad) * kEpiSlotBytes);
     if (lane == 0 && !relay) {
         tma_prefetch_desc(tmO0);
         if (EpiTraits<EPI>::kAct || g.second) tma_prefetch_desc(tmO1);
@@ -969,8 +986,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                     uint32_t acc[32];
                     partial_sum(g, w, nworkers, tile_rows, BN, own_r, c * 32, acc, lane,
                                 sure_last ? w.piece : -1, t_row + c * 32);
-                    epilogue_chunk<EPI>(g, uO, tmO1, acc, tile_row0 + quad * 32, w.nb * BN + c * 32,
-                                        uM, uN, slot, lane, csx, 0, -1);
+                    epilogue_chunk<EPI, DBL>(g, uO, tmO1, acc, tile_row0 + quad * 32, w.nb * BN + c * 32,
+                                             uM, uN, slot, sbuf, lane, csx, 0, -1);
                 }
                 if (sure_last) {
                     // the accumulator was read in the loop above: release it, and
@@ -1036,8 +1053,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 ++xcount;
                 continue;
             }
-            epilogue_chunk<EPI>(g, uO, tmO1, acc, tile_row0 + quad * 32, col0, uM, uN, slot, lane, csx,
-                                cs_on ? 1 : 0, cs_row);
+            epilogue_chunk<EPI, DBL>(g, uO, tmO1, acc, tile_row0 + quad * 32, col0, uM, uN, slot, sbuf,
+                                     lane, csx, cs_on ? 1 : 0, cs_row);
             if constexpr (RELAY) {
                 // the partner relay's chunk: same columns, rows of quad - 2
                 const bool got = mbar_wait_bounded(smem_u32(&xfull[pair_id]), xcount & 1u, abort, limit);
@@ -1056,8 +1073,8 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 }
                 mbar_arrive(smem_u32(&xempty[pair_id]));
                 ++xcount;
-                epilogue_chunk<EPI>(g, uO, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, uM, uN, slot,
-                                    lane, csx, cs_on ? 2 : 0, cs_row);
+                epilogue_chunk<EPI, DBL>(g, uO, tmO1, pacc, tile_row0 + (quad - 2) * 32, col0, uM, uN,
+                                         slot, sbuf, lane, csx, cs_on ? 2 : 0, cs_row);
             }
         }
         if (failed) {

@@ -22,29 +22,39 @@
 
 namespace tpmlp {
 
-template <int BN>
+// DBL: two epilogue staging slots per warp, paid for with one ring stage (5
+// instead of 6).
+template <int BN, bool DBL = false>
 struct Tile2Cfg {
     static_assert(BN == 128 || BN == 256, "pair tiles use BN = 128 or 256");
     static constexpr int A_BYTES = kBM * kBK * 2;         // this CTA's 128 rows
     static constexpr int B_BYTES = (BN / 2) * kBK * 2;    // this CTA's BN/2 columns
     static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;  // per CTA
-    static constexpr int STAGES = (196608 / STAGE_BYTES) > 8 ? 8 : (196608 / STAGE_BYTES);
+    static constexpr int RING_BYTES = DBL ? 163840 : 196608;
+    static constexpr int STAGES = (RING_BYTES / STAGE_BYTES) > 8 ? 8 : (RING_BYTES / STAGE_BYTES);
+    static constexpr int STAGING_BYTES = (DBL ? 2 : 1) * kEpiStagingBytes;
     static constexpr int TMEM_COLS = (2 * BN <= 256) ? 256 : 512;
     // barriers: ring (2·STAGES), accumulators (4), drain, relay (8), item
     // queue (2·kQueue); then the TMEM address, the abort flag, the queue's items
     static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5 + 8 + 2 * kQueue) + 16 + 4 * kQueue;
-    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + kEpiStagingBytes + BAR_BYTES;
+    static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + STAGING_BYTES + BAR_BYTES;
 };
 
 constexpr int kPairM = 2 * kBM;  // 256 rows per pair tile
 
-template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
+// LONG: the variant for long products (bf16 outputs, ≥ 64 k-blocks per tile,
+// ≥ 4 waves of tiles): double epilogue staging (Tile2Cfg's DBL), and the only
+// variant that can run the dynamic schedule (g.dyn_counter non-null). The
+// other variants compile the static schedule alone: a run-time choice between
+// the two in their loops costs the short products (12–24 k-blocks per tile)
+// 6–9% per launch, measured on B200.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY, bool LONG>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_tc2_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                     const __grid_constant__ CUtensorMap tmO0, const __grid_constant__ CUtensorMap tmO1,
                     const __grid_constant__ CUtensorMap tmA2, const __grid_constant__ CUtensorMap tmB2,
                     const GemmArgs g) {
-    using C = Tile2Cfg<BN>;
+    using C = Tile2Cfg<BN, LONG>;
     constexpr int STAGES = C::STAGES;
     constexpr uint32_t IDESC = idesc_bf16_f32(kPairM, BN, A_MN, B_MN);
 
@@ -54,7 +64,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     uint8_t* sA = smem;
     uint8_t* sB = smem + STAGES * C::A_BYTES;
     uint8_t* sEpi = sB + STAGES * C::B_BYTES;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + kEpiStagingBytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sEpi + C::STAGING_BYTES);
     uint64_t* full = bars;
     uint64_t* empty = bars + STAGES;
     uint64_t* tfull = bars + 2 * STAGES;
@@ -89,11 +99,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             mbar_init(smem_u32(&xfull[x]), 32);
             mbar_init(smem_u32(&xempty[x]), 32);
         }
-        // readers of each queue slot: the leader's MMA thread and 8 epilogue
-        // warps, the other CTA's producer and 8 epilogue warps
-        for (int x = 0; x < kQueue; ++x) {
-            mbar_init(smem_u32(&qfull[x]), 1);
-            mbar_init(smem_u32(&qempty[x]), 2 + 2 * kEpiWarps);
+        if constexpr (LONG) {
+            // readers of each queue slot: the leader's MMA thread and 8 epilogue
+            // warps, the other CTA's producer and 8 epilogue warps
+            for (int x = 0; x < kQueue; ++x) {
+                mbar_init(smem_u32(&qfull[x]), 1);
+                mbar_init(smem_u32(&qempty[x]), 2 + 2 * kEpiWarps);
+            }
         }
         *abort = 0;
         fence_mbar_init();
@@ -113,7 +125,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 
     const uint64_t limit = g.wait_limit_ns;  // num_m_blocks counts 256-row blocks
     if (warp == 0) zero_later_counters(g, lane);
-    const bool dyn = g.dyn_counter != nullptr;
+    const bool dyn = LONG && g.dyn_counter != nullptr;  // constant false in the other variants
     const PairQueue queue{smem_u32(qitems), smem_u32(qfull), smem_u32(qempty), leader};
 
     if (warp == 0) {
@@ -277,7 +289,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ------------------------------------------------ epilogue warps (both CTAs)
-        epilogue_role<BN, EPI, true, RELAY>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
+        epilogue_role<BN, EPI, true, RELAY, LONG>(g, &tmO0, &tmO1, tmem_base, tfull, tempty, xfull, xempty, sEpi,
                                             pair, npairs, kPairM, static_cast<int>(rank) * kBM, abort,
                                             limit, warp, lane, dyn ? &queue : nullptr);
     }

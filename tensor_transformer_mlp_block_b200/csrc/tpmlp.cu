@@ -43,15 +43,15 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_split_policy{0};
 std::atomic<bool> g_overlap{true};  // programmatic dependent launches
-std::atomic<bool> g_dynamic{true};  // dynamic tile schedule for long products
+std::atomic<bool> g_dynamic{false};  // dynamic tile schedule for long products (opt-in)
 
 struct DeviceInfo {
     bool init = false;
     int cc_major = 0;
     int num_sms = 0;
-    uint64_t attr_set = 0;       // bit per one-CTA tensor-core kernel instantiation
-    uint64_t attr_set_pair = 0;  // bit per CTA-pair kernel instantiation
-    int max_pairs[64] = {};      // co-resident CTA pairs per pair-kernel instantiation
+    bool attr_set[128] = {};       // per one-CTA tensor-core kernel instantiation
+    bool attr_set_pair[128] = {};  // per CTA-pair kernel instantiation
+    int max_pairs[128] = {};       // co-resident CTA pairs per pair-kernel instantiation
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mutex;
@@ -239,11 +239,11 @@ tpmlp_status timed(int kind, double flops, double bytes, cudaStream_t st, Fn&& f
 
 // ------------------------------------------------------ tensor-core launches
 
-// Index of a tensor-core kernel instantiation (0..47) for per-device caches.
-template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
+// Index of a tensor-core kernel instantiation (0..95) for per-device caches.
+template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY, bool LONG = false>
 constexpr int kernel_id() {
     static_assert(BN == 256, "the launchers use 256-column tiles");
-    return (EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2 + (RELAY ? 1 : 0);
+    return ((EPI * 4 + (A_MN ? 2 : 0) + (B_MN ? 1 : 0)) * 2 + (RELAY ? 1 : 0)) * 2 + (LONG ? 1 : 0);
 }
 
 // How a GEMM launch cuts its work into units (see next_unit).
@@ -333,11 +333,11 @@ tpmlp_status gemm_tc_launch(const void* Aop, const void* Bop, int M, int N, int 
         int devn = 0;
         if (cudaGetDevice(&devn) != cudaSuccess || devn < 0 || devn >= kMaxDevices)
             return TPMLP_ERR_CUDA;
-        if (!(g_dev[devn].attr_set & (uint64_t(1) << id))) {
+        if (!g_dev[devn].attr_set[id]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Cfg::SMEM_BYTES) != cudaSuccess)
                 return TPMLP_ERR_CUDA;
-            g_dev[devn].attr_set |= uint64_t(1) << id;
+            g_dev[devn].attr_set[id] = true;
         }
     }
     const int grid = resolve_sched(g, req, dev->num_sms, kSplittable<EPI, RELAY>);
@@ -355,11 +355,13 @@ struct SecondProduct {
 };
 
 // Same product on CTA pairs: 256 × BN tiles, grid = 2 × (co-resident pairs).
-template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
+// LONG: the long-product variant (double epilogue staging; the only one that
+// runs the dynamic schedule: other variants run req's schedule statically).
+template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY, bool LONG = false>
 tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int K,
                              const SchedReq& req, GemmArgs g, cudaStream_t st,
                              const SecondProduct* second = nullptr) {
-    using Cfg = Tile2Cfg<BN>;
+    using Cfg = Tile2Cfg<BN, LONG>;
     const DeviceInfo* dev = device_info();
     if (dev == nullptr) return TPMLP_ERR_CUDA;
     CUtensorMap tmA, tmB;
@@ -389,8 +391,8 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
     g.num_n_blocks = (N + BN - 1) / BN;
     g.k_blocks = (K + kBK - 1) / kBK;
     g.wait_limit_ns = g_wait_limit_ns.load();
-    auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, RELAY>;
-    constexpr int id = kernel_id<BN, A_MN, B_MN, EPI, RELAY>();
+    auto kern = gemm_tc2_kernel<BN, A_MN, B_MN, EPI, RELAY, LONG>;
+    constexpr int id = kernel_id<BN, A_MN, B_MN, EPI, RELAY, LONG>();
     int max_pairs = 0;
     {
         std::lock_guard<std::mutex> lock(g_dev_mutex);
@@ -398,7 +400,7 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
         if (cudaGetDevice(&devn) != cudaSuccess || devn < 0 || devn >= kMaxDevices)
             return TPMLP_ERR_CUDA;
         DeviceInfo& d = g_dev[devn];
-        if (!(d.attr_set_pair & (uint64_t(1) << id))) {
+        if (!d.attr_set_pair[id]) {
             if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      Cfg::SMEM_BYTES) != cudaSuccess)
                 return TPMLP_ERR_CUDA;
@@ -416,13 +418,13 @@ tpmlp_status gemm_tc2_launch(const void* Aop, const void* Bop, int M, int N, int
             int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess || n < 1) return TPMLP_ERR_CUDA;
             d.max_pairs[id] = n;
-            d.attr_set_pair |= uint64_t(1) << id;
+            d.attr_set_pair[id] = true;
         }
         max_pairs = d.max_pairs[id];
     }
     // never more workers than the plan sized the workspace for (num_sms / 2)
     const int pairs = resolve_sched(g, req, std::min(max_pairs, dev->num_sms / 2), kSplittable<EPI, RELAY>);
-    if (!req.dyn) g.dyn_counter = nullptr;
+    if (!LONG || !req.dyn) g.dyn_counter = nullptr;
     return launch_dep(kern, dim3(2 * pairs), dim3(kThreads), Cfg::SMEM_BYTES, st, tmA, tmB, tmO0, tmO1,
                       tmA2, tmB2, g);
 }
@@ -446,11 +448,33 @@ double gemm_bytes(double M, double N, double K) {
 // K = 2048, 0.033 -> 0.053 ms at K = 768; fp32 store 0.318 -> 0.299 ms at
 // K = 2048; bias store 0.548 -> 0.543 ms at K = 4096, 0.021 -> 0.027 ms at
 // K = 768.
+// The long-product kernel variant (two epilogue staging slots per warp, paid
+// with one ring stage; able to run the dynamic schedule) for a bf16-output
+// product on CTA pairs of at least 64 k-blocks per tile and 4 waves of tiles.
+// Measured on B200 (same runs alternating): double staging is 1.5–3.5% faster
+// for every such product of the 7B- and 175B-class workloads, and 6–15% slower
+// for the GPT-2-small and 350M ones (12–64 k-blocks, 0.6–5 waves), where the
+// producer's look-ahead across short tiles needs the sixth stage.
+int plan_num_sms();
+
+bool long_product(int epi, int64_t M, int64_t N, int64_t K) {
+    if (epi == EPI_F32 || M <= kBM) return false;
+    if (epi == EPI_F32) return false;
+    const int64_t tiles = ((int64_t(M) + kPairM - 1) / kPairM) * ((int64_t(N) + 255) / 256);
+    return (K + kBK - 1) / kBK >= 64 && tiles >= 4 * (plan_num_sms() / 2);
+}
+
 template <int BN, bool A_MN, bool B_MN, int EPI, bool RELAY>
 tpmlp_status gemm_tc_pick(const void* Aop, const void* Bop, int M, int N, int K, const SchedReq& req,
                           const GemmArgs& g, cudaStream_t st) {
     // CTA pairs whenever a 256-row tile is not mostly padding
-    if (M > kBM) return gemm_tc2_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, req, g, st);
+    if (M > kBM) {
+        if constexpr (EPI != EPI_F32) {
+            if (long_product(EPI, M, N, K))
+                return gemm_tc2_launch<BN, A_MN, B_MN, EPI, RELAY, true>(Aop, Bop, M, N, K, req, g, st);
+        }
+        return gemm_tc2_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, req, g, st);
+    }
     return gemm_tc_launch<BN, A_MN, B_MN, EPI, RELAY>(Aop, Bop, M, N, K, req, g, st);
 }
 
@@ -479,16 +503,14 @@ tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, i
 template <int BN, bool A_MN, bool B_MN>
 tpmlp_status gemm_tc_grouped(int kind, const void* A0, const void* B0, int M0, int N0, void* out0,
                              const void* A1, const void* B1, int M1, int N1, void* out1, int K,
-                             int* dyn_counter, cudaStream_t st) {
+                             cudaStream_t st) {
     const double flops = 2.0 * (double(M0) * N0 + double(M1) * N1) * K;
     const double bytes = gemm_bytes<EPI_F32>(M0, N0, K) + gemm_bytes<EPI_F32>(M1, N1, K);
     return timed(kind, flops, bytes, st, [&] {
         GemmArgs g{};
         g.out0 = out0;
         g.ld_out = N0;
-        g.dyn_counter = dyn_counter;
-        SchedReq req;
-        req.dyn = dyn_counter != nullptr;
+        const SchedReq req;  // whole tiles, static (fp32 outputs: no long-product variant)
         const SecondProduct second{A1, B1, M1, N1, out1};
         if (K < kRelayMinKPlain)
             return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, false>(A0, B0, M0, N0, K, req, g, st,
@@ -534,14 +556,16 @@ struct SplitSpace {
 // its count of finished pairs (zero at every launch; the last pair resets them).
 constexpr size_t kDynCounterInts = 2;
 
-// Whether a product runs the dynamic schedule: on CTA pairs (M > 128), with
-// at least 4 waves of items and at least 192 k-blocks per tile. Measured on
-// B200 (same run, alternating): 1.5–2% faster for the 175B-class products
-// with 192–768 k-blocks per tile; no gain with 64–256 (7B-class), and 6%
-// slower with 32 (the 175B-class weight gradients: each item's hand-off
-// costs a fixed time that a short tile does not amortise).
-bool wants_dynamic(int64_t M, int64_t items, int64_t K, int num_sms) {
-    return g_dynamic.load() && M > kBM && items >= 4 * (num_sms / 2) && (K + kBK - 1) / kBK >= 192;
+// Whether a product runs the dynamic schedule: a long product (long_product,
+// the only kernel variant that carries it) with at least 4 waves of items and
+// at least 192 k-blocks per tile. Measured on B200 (same run, alternating):
+// 1.5–2% faster for the 175B-class products with 192–768 k-blocks per tile;
+// no gain with 64–256 (7B-class), and 6% slower with 32 (the 175B-class
+// weight gradients: each item's hand-off costs a fixed time that a short
+// tile does not amortise).
+bool wants_dynamic(int epi, int64_t M, int64_t N, int64_t items, int64_t K, int num_sms) {
+    return g_dynamic.load() && long_product(epi, M, N, K) && items >= 4 * (num_sms / 2) &&
+           (K + kBK - 1) / kBK >= 192;
 }
 
 int64_t pair_tiles(int64_t M, int64_t N) { return ((M + kPairM - 1) / kPairM) * ((N + 255) / 256); }
@@ -630,17 +654,12 @@ bool make_plan(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, Plan* pl)
         auto items = [&](const SchedReq& r, int64_t M, int64_t N) {
             return pair_tiles(M, N) * (r.kind == SCHED_GROUPS ? r.groups : 1);
         };
-        pl->f1.dyn = wants_dynamic(T, items(pl->f1, T, F), h, sms);
-        pl->f2.dyn = wants_dynamic(T, items(pl->f2, T, h), F, sms);
-        pl->b2.dyn = wants_dynamic(T, items(pl->b2, T, F), h, sms);
-        if (pl->group34) {
-            pl->b3.dyn = pl->b4.dyn =
-                wants_dynamic(std::min(F, h), pair_tiles(F, h) + pair_tiles(h, F), T, sms);
-        } else {
-            pl->b3.dyn = wants_dynamic(F, items(pl->b3, F, h), T, sms);
-            pl->b4.dyn = wants_dynamic(h, items(pl->b4, h, F), T, sms);
-        }
-        pl->b5.dyn = wants_dynamic(T, items(pl->b5, T, h), F, sms);
+        pl->f1.dyn = wants_dynamic(EPI_GELU, T, F, items(pl->f1, T, F), h, sms);
+        pl->f2.dyn = wants_dynamic(EPI_BIAS, T, h, items(pl->f2, T, h), F, sms);
+        pl->b2.dyn = wants_dynamic(EPI_DGELU, T, F, items(pl->b2, T, F), h, sms);
+        // the weight gradients (fp32 outputs) always run statically
+        pl->b3.dyn = pl->b4.dyn = false;
+        pl->b5.dyn = wants_dynamic(EPI_BIAS, T, h, items(pl->b5, T, h), F, sms);
         pl->fwd_dyn = pl->f1.dyn || pl->f2.dyn;
         pl->bwd_dyn = pl->b2.dyn || pl->b3.dyn || pl->b4.dyn || pl->b5.dyn;
     }
@@ -1068,17 +1087,15 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // Same kernel and K = T: one launch of both when both run whole tiles.
         if (pl.group34) {
             TPMLP_TRY((gemm_tc_grouped<256, true, true>(K_B34, Y, dZ, iF, ih, dB, X, dH, ih, iF, dA,
-                                                        iT, pl.b3.dyn ? dyn : nullptr, st)));
+                                                        iT, st)));
         } else {
             GemmArgs g3{};
             set_split_space(g3, workspace, pl.off_part, pl.off_ctr);
-            g3.dyn_counter = dyn;
             g3.out0 = dB;
             g3.ld_out = h;
             TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B3, Y, dZ, iF, ih, iT, pl.b3, g3, st)));
             GemmArgs g4{};
             set_split_space(g4, workspace, pl.off_part, pl.off_ctr);
-            g4.dyn_counter = dyn;
             g4.out0 = dA;
             g4.ld_out = F;
             TPMLP_TRY((gemm_tc<256, true, true, EPI_F32>(K_B4, X, dH, ih, iF, iT, pl.b4, g4, st)));

@@ -144,15 +144,36 @@ def test_workspace_size_formula(lib):
         assert binding.plan_schedules(T, h, F, p)["F1"] == binding.SCHED_STREAMK
         assert binding.workspace_size(T, h, F, p) == (_r256(2 * 74 * 256 * 256 * 4)
                                                       + _r256(74 * 16 * 4) + _colsums(T, h, F))
-        # the dynamic schedule (products of ≥ 4 waves on CTA pairs) adds its two
-        # int counters after the split counters
+        # the dynamic schedule, when on, adds its two int counters after the
+        # split counters for bf16-output products of ≥ 4 waves on CTA pairs
+        # and ≥ 192 k-blocks (7B-class: Y·B and dH·Aᵀ, K = 16384)
         binding.set_split_policy(1)
         binding.set_dynamic_schedule(True)
         assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20 + 256
         assert binding.workspace_size(4096, 768, 3072, 2) == _colsums(4096, 768, 3072)  # < 4 waves
+        # only the weight gradients (fp32 outputs; K = T = 12288, 18 × 18
+        # tiles each) would qualify here: they always run statically
+        assert binding.workspace_size(12288, 4608, 4608, 1) == _colsums(12288, 4608, 4608)
     finally:
         binding.set_split_policy(0)
+        binding.set_dynamic_schedule(False)
+
+
+def test_dynamic_schedule_is_opt_in(lib):
+    """Off unless asked for: a call then reserves no dynamic counters (here
+    the 7B-class step on whole tiles, whose Y·B and dH·Aᵀ would qualify)."""
+    from tensor_transformer_mlp_block_b200 import binding
+    assert not binding.get_dynamic_schedule()
+    T, h, F, p = 8192, 4096, 16384, 2
+    binding.set_split_policy(1)
+    try:
+        off = binding.workspace_size(T, h, F, p)
         binding.set_dynamic_schedule(True)
+        assert binding.get_dynamic_schedule()
+        assert binding.workspace_size(T, h, F, p) - off == 256
+    finally:
+        binding.set_dynamic_schedule(False)
+        binding.set_split_policy(0)
 
 
 def test_automatic_schedules_for_the_named_workloads(lib):

@@ -22,9 +22,12 @@ SHAPE = (2000, 12296, 12288, 4)
 
 
 @pytest.fixture(autouse=True)
-def _restore():
-    yield
+def _dynamic_on():
+    """Every test here runs with the schedule on (it is off by default) and
+    puts the defaults back afterwards."""
     binding.set_dynamic_schedule(True)
+    yield
+    binding.set_dynamic_schedule(False)
     binding.set_split_policy(0)
 
 
@@ -105,7 +108,7 @@ def test_dynamic_graph_replay():
 def test_dynamic_plan_reserves_its_counters():
     binding.set_split_policy(0)
     T, h, F, p = SHAPE
-    assert binding.get_dynamic_schedule()
+    assert binding.get_dynamic_schedule()  # set by the fixture
     ws_dyn = binding.workspace_size(T, h, F, p)
     binding.set_dynamic_schedule(False)
     # the dynamic counters share a 256-byte block with the split counters
