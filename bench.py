@@ -563,6 +563,19 @@ def e2e_measure(args, cfg, inp, d, H, Y, Z, gout, ws, p, T, h, dt, dev, stream, 
                     "gradients stay resident"}
 
 
+SCHED_NAMES = {0: "whole tiles", 1: "shard groups", 2: "stream-K tail"}
+
+
+def plan_summary(T, h, F, p, dtype_name):
+    """The work schedule the library plans for each of the six products."""
+    from tensor_transformer_mlp_block_b200 import binding
+    from tensor_transformer_mlp_block_b200.inputs import torch_dtype
+    dt = torch_dtype(dtype_name)
+    kinds = binding.plan_schedules(T, h, F, p, dt)
+    dyn = binding.plan_dynamic(T, h, F, p, dt)
+    return {k: SCHED_NAMES[v] + (", dynamic" if dyn[k] else "") for k, v in kinds.items()}
+
+
 def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, launches, clocks,
           working_set, flops_per_step, T, h, F, p, seconds):
     workload = f"{cfg.name}-class TP-MLP fwd+bwd"
@@ -587,6 +600,7 @@ def _line(args, cfg, world, agg, peaks, peaks_src, roofline, per_kernel, e2e, la
                    "cuda_graph": bool(args.graph), "activation": args.activation,
                    "launch_overlap": args.launch_overlap == "on",
                    "split_policy": args.split_policy,
+                   "schedules": plan_summary(T, h, F, p, cfg.dtype) if args.block == "mlp" else None,
                    "l2": f"working set {working_set / 2**30:.2f} GiB > L2 {L2_BYTES / 2**20:.0f} MiB "
                          "(inputs larger than L2; no flush)"},
         "frac_of_peak": {"measured_burst": agg["value"] / world / peaks["bf16_tflops"],

@@ -216,19 +216,21 @@ int tpmlp_get_split_policy(void);
 void tpmlp_set_launch_overlap(int on);
 int tpmlp_get_launch_overlap(void);
 
-/* Dynamic tile schedule (default off). The SMs of a GPU do not all run a
+/* Dynamic tile schedule (default on). The SMs of a GPU do not all run a
  * tile in the same time (measured on B200: the slowest CTA pairs take ~5%
  * longer, the same pairs in every product), so with a static round-robin of
  * tiles a long product ends with its slowest pair. With this on, the
  * tensor-core products with bf16 outputs that run at least 4 waves of tiles
- * on CTA pairs and at least 192 k-blocks (12288 of K) per tile hand their
- * tiles (and their stream-K segments) out in order from a counter in the
- * workspace: faster pairs take more. Which pair computes a tile does not
- * change the arithmetic: results are bit-identical with it on or off.
- * A call that uses it zeroes its counters with one small kernel first.
- * Off by default: a launch alone runs 2–3% faster with it, but a full
- * forward + backward step, which runs at the GPU's power limit, did not get
- * faster (measured on B200, alternating runs). */
+ * on CTA pairs, at least 192 k-blocks (12288 of K) per tile and at least
+ * 3072 k-blocks of work per CTA pair hand their tiles (and their stream-K
+ * segments) out in order from a counter in the workspace: faster pairs take
+ * more, and the pairs that share an operand panel stay closer together in
+ * time (fewer DRAM re-reads). Which pair computes a tile does not change the
+ * arithmetic: results are bit-identical with it on or off. A call that uses
+ * it zeroes its counters with one small kernel first. (Measured on B200 in
+ * power-limited full steps: the 175B-class step, ~3990 k-blocks per pair,
+ * 0.5% faster; the 7B-class row products, ~1770, 0.7% slower each with it;
+ * hence the thresholds.) */
 void tpmlp_set_dynamic_schedule(int on);
 int tpmlp_get_dynamic_schedule(void);
 
@@ -348,6 +350,13 @@ int64_t tpmlp_schedule_units(int sched, int m_blocks, int n_blocks, int k_blocks
  * under the current split policy, on the current device (148 SMs when no
  * device is present). Writes 6 ints to `kinds`. */
 tpmlp_status tpmlp_plan_schedules(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, int* kinds);
+
+/* Diagnostic, host only: for the same six products in the same order,
+ * whether each runs the dynamic tile schedule (1) or a static one (0), under
+ * the current split policy and tpmlp_set_dynamic_schedule setting, on the
+ * current device (148 SMs when no device is present). Writes 6 ints to
+ * `dyn`. */
+tpmlp_status tpmlp_plan_dynamic(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, int* dyn);
 
 /* Library version, major·10000 + minor·100 + patch. */
 int tpmlp_version(void);

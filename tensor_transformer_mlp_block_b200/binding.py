@@ -30,7 +30,8 @@ EXPORTS = (
     "tpmlp_set_wait_limit_ns", "tpmlp_wait_selftest", "tpmlp_launch_count", "tpmlp_eval_activation",
     "tpmlp_profile_enable", "tpmlp_profile_collect", "tpmlp_profile_kinds", "tpmlp_profile_name",
     "tpmlp_profile_read", "tpmlp_profile_reset", "tp_mlp_bwd_noalloc",
-    "tpmlp_noalloc_scratch_bytes", "tpmlp_schedule_units", "tpmlp_plan_schedules", "tpmlp_version",
+    "tpmlp_noalloc_scratch_bytes", "tpmlp_schedule_units", "tpmlp_plan_schedules", "tpmlp_plan_dynamic",
+    "tpmlp_version",
 )
 
 _lib = None
@@ -61,6 +62,8 @@ def lib() -> ctypes.CDLL:
             L.tpmlp_schedule_units.restype = i64
             L.tpmlp_plan_schedules.argtypes = [i64, i64, i64, ci, ci, ctypes.POINTER(ci)]
             L.tpmlp_plan_schedules.restype = ci
+            L.tpmlp_plan_dynamic.argtypes = [i64, i64, i64, ci, ci, ctypes.POINTER(ci)]
+            L.tpmlp_plan_dynamic.restype = ci
             L.tp_mlp_fwd.argtypes = [vp] * 8 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
             L.tp_mlp_fwd.restype = ctypes.c_int
             L.tp_mlp_bwd.argtypes = [vp] * 12 + [i64, i64, i64, ctypes.c_int, ctypes.c_int, vp, sz, vp]
@@ -474,3 +477,12 @@ def plan_schedules(T: int, h: int, F: int, p: int, dtype: torch.dtype = torch.bf
     code = BF16 if dtype == torch.bfloat16 else FP32
     _check(lib().tpmlp_plan_schedules(T, h, F, p, code, kinds), "tpmlp_plan_schedules")
     return dict(zip(("F1", "F2", "B2", "B3", "B4", "B5"), list(kinds)))
+
+
+def plan_dynamic(T: int, h: int, F: int, p: int, dtype: torch.dtype = torch.bfloat16):
+    """Which of F1, F2, B2, B3, B4, B5 run the dynamic tile schedule at these
+    sizes under the current settings (host only)."""
+    dyn = (ctypes.c_int * 6)()
+    code = BF16 if dtype == torch.bfloat16 else FP32
+    _check(lib().tpmlp_plan_dynamic(T, h, F, p, code, dyn), "tpmlp_plan_dynamic")
+    return dict(zip(("F1", "F2", "B2", "B3", "B4", "B5"), [bool(x) for x in dyn]))

@@ -43,7 +43,7 @@ std::atomic<uint64_t> g_launches{0};
 std::atomic<uint64_t> g_wait_limit_ns{kDefaultWaitLimitNs};
 std::atomic<int> g_split_policy{0};
 std::atomic<bool> g_overlap{true};  // programmatic dependent launches
-std::atomic<bool> g_dynamic{false};  // dynamic tile schedule for long products (opt-in)
+std::atomic<bool> g_dynamic{true};  // dynamic tile schedule for the longest products
 
 struct DeviceInfo {
     bool init = false;
@@ -556,19 +556,30 @@ struct SplitSpace {
 // its count of finished pairs (zero at every launch; the last pair resets them).
 constexpr size_t kDynCounterInts = 2;
 
-// Whether a product runs the dynamic schedule: a long product (long_product,
-// the only kernel variant that carries it) with at least 4 waves of items and
-// at least 192 k-blocks per tile. Measured on B200 (same run, alternating):
-// 1.5–2% faster for the 175B-class products with 192–768 k-blocks per tile;
-// no gain with 64–256 (7B-class), and 6% slower with 32 (the 175B-class
-// weight gradients: each item's hand-off costs a fixed time that a short
-// tile does not amortise).
-bool wants_dynamic(int epi, int64_t M, int64_t N, int64_t items, int64_t K, int num_sms) {
-    return g_dynamic.load() && long_product(epi, M, N, K) && items >= 4 * (num_sms / 2) &&
-           (K + kBK - 1) / kBK >= 192;
-}
-
 int64_t pair_tiles(int64_t M, int64_t N) { return ((M + kPairM - 1) / kPairM) * ((N + 255) / 256); }
+
+// Whether a product runs the dynamic schedule: a long product (long_product,
+// the only kernel variant that carries it) with at least 4 waves of items,
+// at least kDynMinTileKBlocks k-blocks per tile (each item's hand-off costs
+// a fixed time: 6% slower at 32 k-blocks, launches timed alone) and at least
+// kDynMinPairKBlocks k-blocks of work per CTA pair. The last one is where
+// the schedule pays: under a static round-robin the pairs drift apart in
+// proportion to the work each runs (the slowest take ~5% longer per tile),
+// and pairs that share an operand panel then read it from DRAM more than
+// once. Measured on B200 in forward + backward steps of 1.7 s at the power
+// limit (alternating runs, on against off): 175B-class, ~3990 k-blocks per
+// pair in all four row products: step 0.5% faster, DRAM reads of X·A 40%
+// lower (ncu); 7B-class Y·B and dH·Aᵀ, ~1770 k-blocks per pair: 0.7% slower
+// each.
+constexpr int64_t kDynMinTileKBlocks = 192;
+constexpr int64_t kDynMinPairKBlocks = 3072;
+
+bool wants_dynamic(int epi, int64_t M, int64_t N, int64_t items, int64_t K, int num_sms) {
+    const int64_t kb = (K + kBK - 1) / kBK;
+    const int64_t pairs = num_sms / 2;
+    return g_dynamic.load() && long_product(epi, M, N, K) && items >= 4 * pairs &&
+           kb >= kDynMinTileKBlocks && pair_tiles(M, N) * kb >= kDynMinPairKBlocks * pairs;
+}
 
 // Schedule of one tensor-core product (M × N output, K deep) under the
 // current policy (tpmlp_set_split_policy):
@@ -1438,6 +1449,14 @@ tpmlp_status tpmlp_plan_schedules(int64_t T, int64_t h, int64_t F, int p, tpmlp_
     if (kinds == nullptr || !make_plan(T, h, F, p, dt, &pl)) return TPMLP_ERR_INVALID;
     const SchedReq* r[6] = {&pl.f1, &pl.f2, &pl.b2, &pl.b3, &pl.b4, &pl.b5};
     for (int i = 0; i < 6; ++i) kinds[i] = r[i]->kind;
+    return TPMLP_OK;
+}
+
+tpmlp_status tpmlp_plan_dynamic(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt, int* dyn) {
+    Plan pl;
+    if (dyn == nullptr || !make_plan(T, h, F, p, dt, &pl)) return TPMLP_ERR_INVALID;
+    const SchedReq* r[6] = {&pl.f1, &pl.f2, &pl.b2, &pl.b3, &pl.b4, &pl.b5};
+    for (int i = 0; i < 6; ++i) dyn[i] = r[i]->dyn ? 1 : 0;
     return TPMLP_OK;
 }
 

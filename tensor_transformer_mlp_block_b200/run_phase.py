@@ -87,6 +87,7 @@ def main(argv=None) -> None:
     print(json.dumps({"workload": cfg.name, "T": T, "h": h, "F": F, "p": p, "phase": args.phase,
                       "ms_per_step": ms, "tflops": flops / ms / 1e9,
                       "schedules": binding.plan_schedules(T, h, F, p, dt),
+                      "dynamic": binding.plan_dynamic(T, h, F, p, dt),
                       "device_bytes": torch.cuda.max_memory_allocated(dev)}))
 
 

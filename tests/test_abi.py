@@ -145,34 +145,41 @@ def test_workspace_size_formula(lib):
         assert binding.workspace_size(T, h, F, p) == (_r256(2 * 74 * 256 * 256 * 4)
                                                       + _r256(74 * 16 * 4) + _colsums(T, h, F))
         # the dynamic schedule, when on, adds its two int counters after the
-        # split counters for bf16-output products of ≥ 4 waves on CTA pairs
-        # and ≥ 192 k-blocks (7B-class: Y·B and dH·Aᵀ, K = 16384)
+        # split counters for bf16-output products of ≥ 4 waves on CTA pairs,
+        # ≥ 192 k-blocks per tile and ≥ 3072 per pair (here Y·B and dH·Aᵀ,
+        # K = F = 32768: 512 tiles × 512 k-blocks over 74 pairs)
         binding.set_split_policy(1)
         binding.set_dynamic_schedule(True)
-        assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20 + 256
+        assert binding.workspace_size(8192, 4096, 32768, 2) == _colsums(8192, 4096, 32768) + 256
+        assert binding.workspace_size(8192, 4096, 16384, 2) == 9 * 2 ** 20  # 1771 per pair
         assert binding.workspace_size(4096, 768, 3072, 2) == _colsums(4096, 768, 3072)  # < 4 waves
-        # only the weight gradients (fp32 outputs; K = T = 12288, 18 × 18
+        # only the weight gradients (fp32 outputs; K = T = 24576, 18 × 18
         # tiles each) would qualify here: they always run statically
-        assert binding.workspace_size(12288, 4608, 4608, 1) == _colsums(12288, 4608, 4608)
+        assert binding.workspace_size(24576, 4608, 4608, 1) == _colsums(24576, 4608, 4608)
+        # X·A and dZ·Bᵀ with 192 k-blocks per tile and 32 × 16 tiles (6.9
+        # waves), but 1328 k-blocks per pair: static
+        assert binding.workspace_size(8192, 12288, 4096, 2) == _colsums(8192, 12288, 4096)
     finally:
         binding.set_split_policy(0)
-        binding.set_dynamic_schedule(False)
+        binding.set_dynamic_schedule(True)
 
 
-def test_dynamic_schedule_is_opt_in(lib):
-    """Off unless asked for: a call then reserves no dynamic counters (here
-    the 7B-class step on whole tiles, whose Y·B and dH·Aᵀ would qualify)."""
+def test_dynamic_schedule_default(lib):
+    """On by default, for the longest products only: the 7B-class step (~1770
+    k-blocks per CTA pair) reserves no dynamic counters, a step with K = F =
+    32768 (~3540 per pair) does, and switching it off drops them."""
     from tensor_transformer_mlp_block_b200 import binding
-    assert not binding.get_dynamic_schedule()
-    T, h, F, p = 8192, 4096, 16384, 2
+    assert binding.get_dynamic_schedule()
     binding.set_split_policy(1)
     try:
-        off = binding.workspace_size(T, h, F, p)
-        binding.set_dynamic_schedule(True)
-        assert binding.get_dynamic_schedule()
-        assert binding.workspace_size(T, h, F, p) - off == 256
-    finally:
+        on_7b = binding.workspace_size(8192, 4096, 16384, 2)
+        on_long = binding.workspace_size(8192, 4096, 32768, 2)
         binding.set_dynamic_schedule(False)
+        assert not binding.get_dynamic_schedule()
+        assert binding.workspace_size(8192, 4096, 16384, 2) == on_7b
+        assert on_long - binding.workspace_size(8192, 4096, 32768, 2) == 256
+    finally:
+        binding.set_dynamic_schedule(True)
         binding.set_split_policy(0)
 
 
@@ -197,6 +204,30 @@ def test_automatic_schedules_for_the_named_workloads(lib):
     k = binding.plan_schedules(2048, 12288, 49152, 8)
     assert k["F2"] == k["B5"] == binding.SCHED_GROUPS and k["F1"] == TILES
     binding.set_split_policy(0)
+
+
+def test_dynamic_products_of_the_named_workloads(lib):
+    """The dynamic schedule (on by default) takes the four 175B-class row
+    products (~3990 k-blocks per CTA pair each: 1536 tiles of 192 k-blocks,
+    or 384 tiles of 768) and nothing of the smaller workloads (7B-class Y·B
+    and dH·Aᵀ: 512 tiles of 256 k-blocks, ~1770 per pair); never the fp32
+    weight gradients; nothing with it switched off."""
+    import torch
+    from tensor_transformer_mlp_block_b200 import binding
+    binding.set_split_policy(0)
+    assert binding.plan_dynamic(2048, 12288, 49152, 8) == dict(F1=True, F2=True, B2=True, B3=False,
+                                                               B4=False, B5=True)
+    for T, h, F, p in [(8192, 4096, 16384, 2), (4096, 768, 3072, 2), (6144, 1024, 4096, 4)]:
+        assert not any(binding.plan_dynamic(T, h, F, p).values()), (T, h, F, p)
+    assert not any(binding.plan_dynamic(512, 12, 48, 2, torch.float32).values())
+    binding.set_split_policy(2)  # shard groups: the same work per pair, cut finer
+    assert binding.plan_dynamic(2048, 12288, 49152, 8)["F2"]
+    binding.set_split_policy(0)
+    binding.set_dynamic_schedule(False)
+    try:
+        assert not any(binding.plan_dynamic(2048, 12288, 49152, 8).values())
+    finally:
+        binding.set_dynamic_schedule(True)
 
 
 def test_product_path_refuses_cpu_tensors():

@@ -47,3 +47,5 @@ def test_bench_json_line_contract():
     assert d["gpu_launches"] > 0
     assert "sm_mhz" in d["clocks"] and "reasons" in d["clocks"]
     assert "workload" in d["config"]
+    # the planned schedule of each product (GPT-2-small: whole tiles, static)
+    assert d["config"]["schedules"] == {k: "whole tiles" for k in ("F1", "F2", "B2", "B3", "B4", "B5")}

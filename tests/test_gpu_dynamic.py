@@ -13,21 +13,20 @@ from tensor_transformer_mlp_block_b200.inputs import make_shape, sample_indices
 
 pytestmark = pytest.mark.gpu
 
-# the dynamic schedule runs products of ≥ 4 waves of 74 CTA pairs and ≥ 192
-# k-blocks per tile: here X·A and dZ·Bᵀ (K = h = 12296, ragged; 8 × 48 pair
-# tiles), Y·B and dH·Aᵀ (K = F = 12288; 8 × 49 tiles, ragged N) at a ragged
-# token count; the weight gradients (K = T) stay static. F/p = 3072 lets
-# policy 2 cut the row products into shard units.
-SHAPE = (2000, 12296, 12288, 4)
+# the dynamic schedule runs bf16-output products of ≥ 4 waves of 74 CTA
+# pairs, ≥ 192 k-blocks per tile and ≥ 3072 per pair: here X·A and dZ·Bᵀ
+# (K = h = 24584, ragged; 8 × 96 pair tiles), Y·B and dH·Aᵀ (K = F = 24576;
+# 8 × 97 tiles, ragged N), ~4000 k-blocks per pair each, at a ragged token
+# count; the weight gradients (fp32, K = T) stay static.
+# F/p = 6144 lets policy 2 cut the row products into shard units.
+SHAPE = (2000, 24584, 24576, 4)
 
 
 @pytest.fixture(autouse=True)
-def _dynamic_on():
-    """Every test here runs with the schedule on (it is off by default) and
-    puts the defaults back afterwards."""
+def _restore():
     binding.set_dynamic_schedule(True)
     yield
-    binding.set_dynamic_schedule(False)
+    binding.set_dynamic_schedule(True)
     binding.set_split_policy(0)
 
 
@@ -108,7 +107,7 @@ def test_dynamic_graph_replay():
 def test_dynamic_plan_reserves_its_counters():
     binding.set_split_policy(0)
     T, h, F, p = SHAPE
-    assert binding.get_dynamic_schedule()  # set by the fixture
+    assert binding.get_dynamic_schedule()
     ws_dyn = binding.workspace_size(T, h, F, p)
     binding.set_dynamic_schedule(False)
     # the dynamic counters share a 256-byte block with the split counters
