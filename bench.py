@@ -159,7 +159,12 @@ def pick_tensor_peak(peaks: dict, src: str, region_s: float, clocks: dict):
     if region_s >= SUSTAINED_MIN_SECONDS and capped and "bf16_tflops_sustained" in peaks:
         return peaks["bf16_tflops_sustained"], (
             f"{src} bf16 sustained: timed region {region_s:.2f} s under sw_power_cap")
-    why = "short" if region_s < SUSTAINED_MIN_SECONDS else "not power-capped"
+    if region_s < SUSTAINED_MIN_SECONDS:
+        why = "short"
+    elif not capped:
+        why = "not power-capped"
+    else:
+        why = "power-capped, but no sustained figure was measured"
     return peaks["bf16_tflops"], f"{src} bf16 burst: timed region {region_s:.2f} s ({why})"
 
 

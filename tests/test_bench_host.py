@@ -26,6 +26,7 @@ def test_fallback_has_no_sustained_figure():
     assert fb == {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
     peak, src = bench.pick_tensor_peak(fb, "fallback", 5.0, {"reasons": ["sw_power_cap"]})
     assert peak == 1590.0 and src.startswith("fallback bf16 burst")
+    assert "no sustained figure" in src and "not power-capped" not in src
 
 
 def test_default_workload_is_the_largest():
