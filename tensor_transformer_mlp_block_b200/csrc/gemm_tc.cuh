@@ -979,6 +979,18 @@ __device__ __forceinline__ void epilogue_role(const GemmArgs& g, const CUtensorM
                 last = partial_arrive(ctr, w.pieces, lane);
             }
             if (last) {
+                if (RELAY && relay) {
+                    // The slot may still hold the last chunk this warp relayed
+                    // on an earlier whole tile: it is staged over only once the
+                    // partner has taken that chunk (the wait passes at once if
+                    // it has, or if nothing was relayed yet).
+                    const bool got = mbar_wait_bounded(smem_u32(&xempty[pair_id]), (xcount & 1u) ^ 1u,
+                                                       abort, limit);
+                    if (!__all_sync(0xffffffffu, got)) {
+                        raise_timeout(abort);
+                        break;
+                    }
+                }
                 float csx[32];  // unused: no column sums on split tiles
 #pragma unroll 1
                 for (int i = 0; i < kChunks; ++i) {
