@@ -63,13 +63,16 @@ typedef enum tpmlp_dtype { TPMLP_BF16 = 0, TPMLP_FP32 = 1 } tpmlp_dtype;
 typedef enum tpmlp_activation { TPMLP_GELU_ERF = 0, TPMLP_GELU_TANH = 1 } tpmlp_activation;
 
 /* Bytes of device workspace that tp_mlp_fwd and tp_mlp_bwd need for these
- * sizes under the current split policy (the larger of the two calls' needs).
- * Returns 0 for invalid sizes. Holds, each part rounded up to 256 bytes:
- * the fp32 partial tiles and the arrival counters of products whose output
- * tiles are split over several work units (see tpmlp_set_split_policy;
- * none when no product splits), and the partial column sums of the bias
+ * sizes under the current split policy and dynamic-schedule setting (the
+ * larger of the two calls' needs). Returns 0 for invalid sizes. Holds, each
+ * part rounded up to 256 bytes: the fp32 partial tiles and the arrival
+ * counters of products whose output tiles are split over several work units
+ * (see tpmlp_set_split_policy; none when no product splits), followed by the
+ * dynamic schedule's two int counters when some product runs it (see
+ * tpmlp_set_dynamic_schedule), and the partial column sums of the bias
  * gradients. The contents need no initialisation: a call that splits tiles
- * first zeroes the counters itself. */
+ * or runs the dynamic schedule first zeroes the counters itself. Changing
+ * either setting can change the size: query it after setting them. */
 size_t tpmlp_workspace_size(int64_t T, int64_t h, int64_t F, int p, tpmlp_dtype dt);
 
 /* Forward (column-parallel, then row-parallel):
