@@ -483,6 +483,22 @@ tpmlp_status gemm_tc_pick(const void* Aop, const void* Bop, int M, int N, int K,
 constexpr int kRelayMinKAct = 3072;    // GeLU and GeLU′ epilogues
 constexpr int kRelayMinKPlain = 2048;  // bias and fp32 epilogues
 
+// The relay also needs work to hide behind: it keeps the sub-partitions of
+// the producer and the MMA issuer free for the next unit's K loop, but it
+// halves the warps that compute and store, and a pair's last unit's epilogue
+// overlaps nothing. With at most two units per CTA pair (on CTA pairs: M >
+// 128) the full-width epilogue is faster. Measured on B200, alternating runs,
+// bit-identical results: GPT-2-small step 698–709 → 736–742 TFLOP/s (Y·B and
+// dH·Aᵀ, 48 tiles, 7–10% faster; the weight gradients, 72 tiles, 6%), 350M
+// 987–995 → 1002–1012 (96 and 128 tiles, 2–4%); the 7B- and 175B-class
+// products (≥ 512 tiles) keep the relay. The GeLU′ epilogue keeps the K rule
+// alone: its da column sums are fused only into the relaying form.
+bool relay_has_work(int64_t M, int64_t units) {
+    return M <= kBM || units > 2 * static_cast<int64_t>(plan_num_sms() / 2);
+}
+
+int64_t pair_tiles(int64_t M, int64_t N) { return ((M + kPairM - 1) / kPairM) * ((N + 255) / 256); }
+
 template <int BN, bool A_MN, bool B_MN, int EPI>
 tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, int K,
                      const SchedReq& req, GemmArgs g, cudaStream_t st) {
@@ -490,7 +506,8 @@ tpmlp_status gemm_tc(int kind, const void* Aop, const void* Bop, int M, int N, i
         const int k_per_unit = req.kind == SCHED_GROUPS && req.groups > 1 ? K / req.groups : K;
         const int threshold =
             (EpiTraits<EPI>::kAct || EpiTraits<EPI>::kDAct) ? kRelayMinKAct : kRelayMinKPlain;
-        if (k_per_unit < threshold)
+        const int64_t units = pair_tiles(M, N) * (req.kind == SCHED_GROUPS ? req.groups : 1);
+        if (k_per_unit < threshold || (!EpiTraits<EPI>::kDAct && !relay_has_work(M, units)))
             return gemm_tc_pick<BN, A_MN, B_MN, EPI, false>(Aop, Bop, M, N, K, req, g, st);
         return gemm_tc_pick<BN, A_MN, B_MN, EPI, true>(Aop, Bop, M, N, K, req, g, st);
     });
@@ -512,7 +529,7 @@ tpmlp_status gemm_tc_grouped(int kind, const void* A0, const void* B0, int M0, i
         g.ld_out = N0;
         const SchedReq req;  // whole tiles, static (fp32 outputs: no long-product variant)
         const SecondProduct second{A1, B1, M1, N1, out1};
-        if (K < kRelayMinKPlain)
+        if (K < kRelayMinKPlain || !relay_has_work(M0, pair_tiles(M0, N0) + pair_tiles(M1, N1)))
             return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, false>(A0, B0, M0, N0, K, req, g, st,
                                                                  &second);
         return gemm_tc2_launch<BN, A_MN, B_MN, EPI_F32, true>(A0, B0, M0, N0, K, req, g, st,
@@ -555,8 +572,6 @@ struct SplitSpace {
 // Two ints after the split counters: the dynamic schedule's item counter and
 // its count of finished pairs (zero at every launch; the last pair resets them).
 constexpr size_t kDynCounterInts = 2;
-
-int64_t pair_tiles(int64_t M, int64_t N) { return ((M + kPairM - 1) / kPairM) * ((N + 255) / 256); }
 
 // Whether a product runs the dynamic schedule: a long product (long_product,
 // the only kernel variant that carries it) with at least 4 waves of items,
