@@ -1,56 +1,10 @@
-// Bandwidth-bound helper kernels: the ordered sum of split partials (the
-// on-chip counterpart of the all-reduce after the row-parallel product) and
-// deterministic column sums (the bias gradients).
+// Bandwidth-bound helper kernels: deterministic column sums (the bias
+// gradients), the activation rebuild for recompute, and small utilities.
 #pragma once
 
 #include "gemm_tc.cuh"
 
 namespace tpmlp {
-
-// out[m, n] = round( Σ_{s=0..S-1} ws[s][m, n] + bias[n] ), the partials
-// added in ascending s, then the bias once. Each thread handles 8
-// consecutive columns (N % 8 == 0; all pointers 16-byte aligned).
-__global__ void __launch_bounds__(256) reduce_splits_bf16_kernel(
-    const float* __restrict__ ws, int splits, int64_t plane, const __nv_bfloat16* __restrict__ bias,
-    __nv_bfloat16* __restrict__ out, int64_t M, int64_t N) {
-    grid_dep_wait();  // every input may come from the predecessor kernel
-    grid_dep_launch();
-    const int64_t groups = M * (N / 8);
-    for (int64_t gi = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; gi < groups;
-         gi += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-        const int64_t e = gi * 8;
-        float4 lo = __ldg(reinterpret_cast<const float4*>(ws + e));
-        float4 hi = __ldg(reinterpret_cast<const float4*>(ws + e + 4));
-        float v[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-        for (int s = 1; s < splits; ++s) {
-            const float* p = ws + s * plane + e;
-            lo = __ldg(reinterpret_cast<const float4*>(p));
-            hi = __ldg(reinterpret_cast<const float4*>(p + 4));
-            v[0] += lo.x; v[1] += lo.y; v[2] += lo.z; v[3] += lo.w;
-            v[4] += hi.x; v[5] += hi.y; v[6] += hi.z; v[7] += hi.w;
-        }
-        if (bias != nullptr) {
-            const int64_t n = e % N;
-            const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(bias + n);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float2 t = __bfloat1622float2(b2[i]);
-                v[2 * i] += t.x;
-                v[2 * i + 1] += t.y;
-            }
-        }
-        uint4 o;
-        __nv_bfloat162 r0 = __floats2bfloat162_rn(v[0], v[1]);
-        __nv_bfloat162 r1 = __floats2bfloat162_rn(v[2], v[3]);
-        __nv_bfloat162 r2 = __floats2bfloat162_rn(v[4], v[5]);
-        __nv_bfloat162 r3 = __floats2bfloat162_rn(v[6], v[7]);
-        o.x = *reinterpret_cast<uint32_t*>(&r0);
-        o.y = *reinterpret_cast<uint32_t*>(&r1);
-        o.z = *reinterpret_cast<uint32_t*>(&r2);
-        o.w = *reinterpret_cast<uint32_t*>(&r3);
-        *reinterpret_cast<uint4*>(out + e) = o;
-    }
-}
 
 template <typename T>
 __device__ __forceinline__ float to_f32(T v);
@@ -59,20 +13,19 @@ __device__ __forceinline__ float to_f32<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-// Column sums, pass 1. Block (32, 8): lane x covers columns
-// [blockIdx.x·256 + 8x, +8), row phase y walks rows chunk_begin + y, +8, ...
-// of chunk blockIdx.y; the 8 phases are then added in order y = 0..7 and
-// the chunk's sums written to partial[blockIdx.y][:]. Fixed assignment and
-// fixed order: the result is bit-reproducible.
+// Column sums, pass 1, one block's share. Block (32, 8): lane x covers
+// columns [bx·256 + 8x, +8), row phase y walks rows chunk_begin + y, +8, ...
+// of chunk `chunk`; the 8 phases are then added in order y = 0..7 and the
+// chunk's sums written to partial[chunk][:]. Fixed assignment and fixed
+// order: the result is bit-reproducible.
 template <typename T, bool VEC>
-__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ X, int64_t R,
-                                                            int64_t C, int64_t rows_per_chunk,
-                                                            float* __restrict__ partial) {
-    grid_dep_wait();  // every input may come from the predecessor kernel
-    grid_dep_launch();
+__device__ __forceinline__ void colsum_partial_block(const T* __restrict__ X, int64_t R, int64_t C,
+                                                     int64_t rows_per_chunk,
+                                                     float* __restrict__ partial, int64_t bx,
+                                                     int64_t chunk) {
     __shared__ float red[8][256];
-    const int64_t c0 = blockIdx.x * 256 + threadIdx.x * 8;
-    const int64_t r_begin = blockIdx.y * rows_per_chunk;
+    const int64_t c0 = bx * 256 + threadIdx.x * 8;
+    const int64_t r_begin = chunk * rows_per_chunk;
     const int64_t r_end = min(R, r_begin + rows_per_chunk);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (VEC && c0 < C) {
@@ -135,12 +88,40 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
     for (int i = 0; i < 8; ++i) red[threadIdx.y][threadIdx.x * 8 + i] = acc[i];
     __syncthreads();
     const int t = threadIdx.y * 32 + threadIdx.x;  // 0..255: one column each
-    const int64_t c = blockIdx.x * 256 + t;
+    const int64_t c = bx * 256 + t;
     if (c < C) {
         float s = red[0][t];
         for (int y = 1; y < 8; ++y) s += red[y][t];
-        partial[blockIdx.y * C + c] = s;
+        partial[chunk * C + c] = s;
     }
+}
+
+// Pass 1 of one R × C matrix: grid (⌈C/256⌉, chunks).
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict__ X, int64_t R,
+                                                            int64_t C, int64_t rows_per_chunk,
+                                                            float* __restrict__ partial) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
+    colsum_partial_block<T, VEC>(X, R, C, rows_per_chunk, partial, blockIdx.x, blockIdx.y);
+}
+
+// Pass 1 of two matrices with the same R (column blocks of X1 first, then
+// of X2: grid (⌈C1/256⌉ + ⌈C2/256⌉, chunks)); each column's sum is the one
+// colsum_partial_kernel computes.
+template <typename T, bool VEC>
+__global__ void __launch_bounds__(256) colsum_partial2_kernel(const T* __restrict__ X1, int64_t C1,
+                                                             float* __restrict__ partial1,
+                                                             const T* __restrict__ X2, int64_t C2,
+                                                             float* __restrict__ partial2, int64_t R,
+                                                             int64_t rows_per_chunk) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int64_t nb1 = (C1 + 255) / 256;
+    if (blockIdx.x < nb1)
+        colsum_partial_block<T, VEC>(X1, R, C1, rows_per_chunk, partial1, blockIdx.x, blockIdx.y);
+    else
+        colsum_partial_block<T, VEC>(X2, R, C2, rows_per_chunk, partial2, blockIdx.x - nb1, blockIdx.y);
 }
 
 // Column sums, pass 2: out[c] = Σ over chunks of partial[chunk][c]. Block
@@ -148,13 +129,10 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
 // contiguous chunk groups; each thread adds its group's chunks in ascending
 // order, then the 8 group sums are added in ascending group order. Fixed
 // assignment and order: bit-reproducible.
-__global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ partial,
-                                                          int chunks, int64_t C,
-                                                          float* __restrict__ out) {
-    grid_dep_wait();  // every input may come from the predecessor kernel
-    grid_dep_launch();
+__device__ __forceinline__ void colsum_final_block(const float* __restrict__ partial, int chunks,
+                                                   int64_t C, float* __restrict__ out, int64_t bx) {
     __shared__ float grp[8][32];
-    const int64_t c = blockIdx.x * 32 + threadIdx.x;
+    const int64_t c = bx * 32 + threadIdx.x;
     const int per = (chunks + 7) / 8;
     const int k0 = threadIdx.y * per;
     const int k1 = min(chunks, k0 + per);
@@ -178,6 +156,33 @@ __global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restri
         for (int y = 1; y < 8; ++y) t += grp[y][threadIdx.x];
         out[c] = t;
     }
+}
+
+// Pass 2 of one matrix: grid ⌈C/32⌉.
+__global__ void __launch_bounds__(256) colsum_final_kernel(const float* __restrict__ partial,
+                                                          int chunks, int64_t C,
+                                                          float* __restrict__ out) {
+    grid_dep_wait();  // every input may come from the predecessor kernel
+    grid_dep_launch();
+    colsum_final_block(partial, chunks, C, out, blockIdx.x);
+}
+
+// Pass 2 of two matrices (the column blocks of the first, then of the
+// second: grid ⌈C1/32⌉ + ⌈C2/32⌉); each sum is the one colsum_final_kernel
+// computes.
+__global__ void __launch_bounds__(256) colsum_final2_kernel(const float* __restrict__ partial1,
+                                                           int chunks1, int64_t C1,
+                                                           float* __restrict__ out1,
+                                                           const float* __restrict__ partial2,
+                                                           int chunks2, int64_t C2,
+                                                           float* __restrict__ out2) {
+    grid_dep_wait();
+    grid_dep_launch();
+    const int64_t nb1 = (C1 + 31) / 32;
+    if (blockIdx.x < nb1)
+        colsum_final_block(partial1, chunks1, C1, out1, blockIdx.x);
+    else
+        colsum_final_block(partial2, chunks2, C2, out2, blockIdx.x - nb1);
 }
 
 // GeLU and GeLU′ of n values with each form the library uses:

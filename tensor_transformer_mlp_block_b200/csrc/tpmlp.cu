@@ -174,14 +174,14 @@ tpmlp_status launch_dep(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sm
 
 enum Kind : int {
     K_F1 = 0, K_F2, K_B1_DB, K_B2, K_B2_DA, K_B3, K_B4, K_B34, K_B5, K_MISC,
-    K_L_FWD, K_L_DB, K_L_DW, K_L_DX, K_RECOMP, K_CTR, K_COUNT
+    K_L_FWD, K_L_DB, K_L_DW, K_L_DX, K_RECOMP, K_CTR, K_B12, K_COUNT
 };
 const char* const kKindNames[K_COUNT] = {
     "F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum", "B1.db_colsum",
     "B2.dgrad_gelu_grad",    "B2.da_colsum",          "B3.wgrad_dB",     "B4.wgrad_dA",
     "B3+B4.wgrad_dB_dA",     "B5.dgrad_dX_shard_sum", "misc",
     "L.fwd_gemm_bias",       "L.dbias_colsum",        "L.wgrad_dW",      "L.dgrad_dX",
-    "R.recompute_activation", "S.counter_reset",
+    "R.recompute_activation", "S.counter_reset",  "B1+B2.db_da_colsum",
 };
 
 struct KindTotals {
@@ -760,6 +760,30 @@ tpmlp_status colsum(int kind, const T* X, int64_t R, int64_t C, int64_t chunks, 
                  [&] { return colsum_launch(X, R, C, chunks, partial, out, st); });
 }
 
+// Both bias gradients' column sums in two launches instead of four: pass 1
+// over X1 (R × C1) and X2 (R × C2) in one grid, then pass 2 of both. Each
+// column's sum is computed exactly as colsum computes it.
+template <typename T>
+tpmlp_status colsum2(int kind, const T* X1, int64_t C1, float* partial1, float* out1, const T* X2,
+                     int64_t C2, float* partial2, float* out2, int64_t R, int64_t chunks,
+                     cudaStream_t st) {
+    return timed(kind, 0.0, sizeof(T) * double(R) * (C1 + C2) + 4.0 * (C1 + C2), st, [&] {
+        dim3 grid(static_cast<unsigned>((C1 + 255) / 256 + (C2 + 255) / 256),
+                  static_cast<unsigned>(chunks));
+        const bool vec = C1 % 8 == 0 && C2 % 8 == 0 && aligned16(X1) && aligned16(X2);
+        const tpmlp_status s =
+            vec ? launch_dep(colsum_partial2_kernel<T, true>, grid, dim3(32, 8), 0, st, X1, C1,
+                             partial1, X2, C2, partial2, R, kColsumRowsPerChunk)
+                : launch_dep(colsum_partial2_kernel<T, false>, grid, dim3(32, 8), 0, st, X1, C1,
+                             partial1, X2, C2, partial2, R, kColsumRowsPerChunk);
+        if (s != TPMLP_OK) return s;
+        return launch_dep(colsum_final2_kernel,
+                          dim3(static_cast<unsigned>((C1 + 31) / 32 + (C2 + 31) / 32)), dim3(32, 8), 0,
+                          st, static_cast<const float*>(partial1), static_cast<int>(chunks), C1, out1,
+                          static_cast<const float*>(partial2), static_cast<int>(chunks), C2, out2);
+    });
+}
+
 // Pass 2 alone: out[c] = Σ over `rows` partial rows of partial[r][c], in
 // ascending r (partials written by a GEMM epilogue).
 tpmlp_status colsum_finish(int kind, const float* partial, int64_t rows, int64_t C, float* out,
@@ -1084,14 +1108,16 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         const __nv_bfloat16* dZb = static_cast<const __nv_bfloat16*>(dZ);
         int* dyn = dyn_space(workspace, pl.off_dyn);
         if (pl.bwd_dyn) TPMLP_TRY(reset_counters(workspace, pl.off_ctr, pl.ctr_bytes, st));
-        // db = 1ᵀ·dZ
-        TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         // B2: dH = (dZ·Bᵀ) ⊙ GeLU′(H). Aop = dZ [T][h] (K-major), Bop = B [F][h] (K-major).
         // With the relaying epilogue (long K) the computing warps have room to
         // also leave the column sums of dH in cs_f (two partial rows per
         // 128-row tile); da then needs only their ordered sum. With short K
-        // the extra epilogue work costs more than the separate pass.
+        // the extra epilogue work costs more than the separate pass, and db
+        // (which nothing in the backward reads) waits for it: both column
+        // sums then take one two-pass pair of launches after B2.
         const bool fused_da = h >= kRelayMinKAct;
+        // db = 1ᵀ·dZ
+        if (fused_da) TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
         GemmArgs g2{};
         set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
         g2.dyn_counter = dyn;
@@ -1102,12 +1128,12 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         g2.aux = static_cast<const __nv_bfloat16*>(H);
         g2.colsum_out = fused_da ? cs_f : nullptr;
         TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, pl.b2, g2, st)));
-        // da = 1ᵀ·dH
+        // da = 1ᵀ·dH (and db with it where it waited)
         if (fused_da)
             TPMLP_TRY(colsum_finish(K_B2_DA, cs_f, da_partial_rows(T), F, da, st));
         else
-            TPMLP_TRY(colsum(K_B2_DA, static_cast<const __nv_bfloat16*>(dH), T, F, pl.chunks, cs_f,
-                             da, st));
+            TPMLP_TRY(colsum2(K_B12, dZb, h, cs_h, db, static_cast<const __nv_bfloat16*>(dH), F, cs_f,
+                              da, T, pl.chunks, st));
         // B3: dB = Yᵀ·dZ. Aop = Y [T][F] (MN-major, M = F), Bop = dZ [T][h] (MN-major).
         // B4: dA = Xᵀ·dH. Aop = X [T][h] (MN-major, M = h), Bop = dH [T][F] (MN-major).
         // Same kernel and K = T: one launch of both when both run whole tiles.
