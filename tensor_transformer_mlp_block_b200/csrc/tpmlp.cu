@@ -784,13 +784,30 @@ tpmlp_status colsum2(int kind, const T* X1, int64_t C1, float* partial1, float* 
     });
 }
 
-// Pass 2 alone: out[c] = Σ over `rows` partial rows of partial[r][c], in
-// ascending r (partials written by a GEMM epilogue).
-tpmlp_status colsum_finish(int kind, const float* partial, int64_t rows, int64_t C, float* out,
-                           cudaStream_t st) {
-    return timed(kind, 0.0, 4.0 * double(rows) * C + 4.0 * C, st, [&] {
-        return launch_dep(colsum_final_kernel, dim3(static_cast<unsigned>((C + 31) / 32)),
-                          dim3(32, 8), 0, st, partial, static_cast<int>(rows), C, out);
+// Pass 1 alone (its pass 2 runs later through colsum_finish2).
+template <typename T>
+tpmlp_status colsum_first(int kind, const T* X, int64_t R, int64_t C, int64_t chunks, float* partial,
+                          cudaStream_t st) {
+    return timed(kind, 0.0, sizeof(T) * double(R) * C + 4.0 * double(chunks) * C, st, [&] {
+        dim3 grid(static_cast<unsigned>((C + 255) / 256), static_cast<unsigned>(chunks));
+        return (C % 8 == 0 && aligned16(X))
+                   ? launch_dep(colsum_partial_kernel<T, true>, grid, dim3(32, 8), 0, st, X, R, C,
+                                kColsumRowsPerChunk, partial)
+                   : launch_dep(colsum_partial_kernel<T, false>, grid, dim3(32, 8), 0, st, X, R, C,
+                                kColsumRowsPerChunk, partial);
+    });
+}
+
+// Pass 2 of two sets of partials in one launch: out1[c] = Σ_r partial1[r][c]
+// over rows1 rows and out2 likewise, each in ascending r.
+tpmlp_status colsum_finish2(int kind, const float* partial1, int64_t rows1, int64_t C1, float* out1,
+                            const float* partial2, int64_t rows2, int64_t C2, float* out2,
+                            cudaStream_t st) {
+    return timed(kind, 0.0, 4.0 * (double(rows1) * C1 + double(rows2) * C2 + C1 + C2), st, [&] {
+        return launch_dep(colsum_final2_kernel,
+                          dim3(static_cast<unsigned>((C1 + 31) / 32 + (C2 + 31) / 32)), dim3(32, 8), 0,
+                          st, partial1, static_cast<int>(rows1), C1, out1, partial2,
+                          static_cast<int>(rows2), C2, out2);
     });
 }
 
@@ -1114,10 +1131,12 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         // 128-row tile); da then needs only their ordered sum. With short K
         // the extra epilogue work costs more than the separate pass, and db
         // (which nothing in the backward reads) waits for it: both column
-        // sums then take one two-pass pair of launches after B2.
+        // sums then take one two-pass pair of launches after B2. With da
+        // fused, db's first pass runs before B2 and its second shares one
+        // launch with da's ordered sum after it.
         const bool fused_da = h >= kRelayMinKAct;
-        // db = 1ᵀ·dZ
-        if (fused_da) TPMLP_TRY(colsum(K_B1_DB, dZb, T, h, pl.chunks, cs_h, db, st));
+        // db = 1ᵀ·dZ, pass 1
+        if (fused_da) TPMLP_TRY(colsum_first(K_B1_DB, dZb, T, h, pl.chunks, cs_h, st));
         GemmArgs g2{};
         set_split_space(g2, workspace, pl.off_part, pl.off_ctr);
         g2.dyn_counter = dyn;
@@ -1128,9 +1147,9 @@ tpmlp_status bwd_impl(const void* dZ, const void* X, const void* A, const void* 
         g2.aux = static_cast<const __nv_bfloat16*>(H);
         g2.colsum_out = fused_da ? cs_f : nullptr;
         TPMLP_TRY((gemm_tc<256, false, false, EPI_DACT>(K_B2, dZ, B, iT, iF, ih, pl.b2, g2, st)));
-        // da = 1ᵀ·dH (and db with it where it waited)
+        // da = 1ᵀ·dH and db's pass 2 (or both whole column sums)
         if (fused_da)
-            TPMLP_TRY(colsum_finish(K_B2_DA, cs_f, da_partial_rows(T), F, da, st));
+            TPMLP_TRY(colsum_finish2(K_B12, cs_h, pl.chunks, h, db, cs_f, da_partial_rows(T), F, da, st));
         else
             TPMLP_TRY(colsum2(K_B12, dZb, h, cs_h, db, static_cast<const __nv_bfloat16*>(dH), F, cs_f,
                               da, T, pl.chunks, st));
