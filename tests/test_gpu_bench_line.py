@@ -49,3 +49,9 @@ def test_bench_json_line_contract():
     assert "workload" in d["config"]
     # the planned schedule of each product (GPT-2-small: whole tiles, static)
     assert d["config"]["schedules"] == {k: "whole tiles" for k in ("F1", "F2", "B2", "B3", "B4", "B5")}
+    # the step's launch structure at this size: five GEMM launches (B3 and B4
+    # share one) and one two-pass pair for both bias gradients
+    assert d["gpu_launches"] == 7 * d["steps"]
+    assert set(d["kernels"]) == {"F1.col_gemm_bias_gelu", "F2.row_gemm_shard_sum",
+                                 "B2.dgrad_gelu_grad", "B3+B4.wgrad_dB_dA",
+                                 "B5.dgrad_dX_shard_sum", "B1+B2.db_da_colsum"}
