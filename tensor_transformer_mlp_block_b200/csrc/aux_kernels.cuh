@@ -21,19 +21,18 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return
 template <typename T, bool VEC>
 __device__ __forceinline__ void colsum_partial_block(const T* __restrict__ X, int64_t R, int64_t C,
                                                      int64_t rows_per_chunk,
-                                                     float* __restrict__ partial, int64_t bx,
-                                                     int64_t chunk) {
+                                                     float* __restrict__ partial, int bx, int chunk) {
     __shared__ float red[8][256];
-    const int64_t c0 = bx * 256 + threadIdx.x * 8;
-    const int64_t r_begin = chunk * rows_per_chunk;
+    const int64_t c0 = static_cast<int64_t>(bx) * 256 + threadIdx.x * 8;
+    const int64_t r_begin = static_cast<int64_t>(chunk) * rows_per_chunk;
     const int64_t r_end = min(R, r_begin + rows_per_chunk);
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
     if (VEC && c0 < C) {
         // C % 8 == 0 and X 16-byte aligned: 8 columns are 16 (bf16) or 32 (fp32)
         // bytes. Rows are visited in the same order as the scalar loop, but
-        // the loads of up to kU rows are issued before their additions so
-        // that many are in flight at once.
-        constexpr int kU = 8;
+        // the loads of up to kU rows (128 bytes per thread) are issued before
+        // their additions so that many are in flight at once.
+        constexpr int kU = sizeof(T) == 2 ? 8 : 4;
         int64_t r = r_begin + threadIdx.y;
         for (; r + 8 * (kU - 1) < r_end; r += 8 * kU) {
             if constexpr (sizeof(T) == 2) {
@@ -88,11 +87,11 @@ __device__ __forceinline__ void colsum_partial_block(const T* __restrict__ X, in
     for (int i = 0; i < 8; ++i) red[threadIdx.y][threadIdx.x * 8 + i] = acc[i];
     __syncthreads();
     const int t = threadIdx.y * 32 + threadIdx.x;  // 0..255: one column each
-    const int64_t c = bx * 256 + t;
+    const int64_t c = static_cast<int64_t>(bx) * 256 + t;
     if (c < C) {
         float s = red[0][t];
         for (int y = 1; y < 8; ++y) s += red[y][t];
-        partial[chunk * C + c] = s;
+        partial[static_cast<int64_t>(chunk) * C + c] = s;
     }
 }
 
@@ -103,7 +102,8 @@ __global__ void __launch_bounds__(256) colsum_partial_kernel(const T* __restrict
                                                             float* __restrict__ partial) {
     grid_dep_wait();  // every input may come from the predecessor kernel
     grid_dep_launch();
-    colsum_partial_block<T, VEC>(X, R, C, rows_per_chunk, partial, blockIdx.x, blockIdx.y);
+    colsum_partial_block<T, VEC>(X, R, C, rows_per_chunk, partial, static_cast<int>(blockIdx.x),
+                                 static_cast<int>(blockIdx.y));
 }
 
 // Pass 1 of two matrices with the same R (column blocks of X1 first, then
@@ -117,11 +117,12 @@ __global__ void __launch_bounds__(256) colsum_partial2_kernel(const T* __restric
                                                              int64_t rows_per_chunk) {
     grid_dep_wait();
     grid_dep_launch();
-    const int64_t nb1 = (C1 + 255) / 256;
-    if (blockIdx.x < nb1)
-        colsum_partial_block<T, VEC>(X1, R, C1, rows_per_chunk, partial1, blockIdx.x, blockIdx.y);
+    const int nb1 = static_cast<int>((C1 + 255) / 256);
+    const int bx = static_cast<int>(blockIdx.x), by = static_cast<int>(blockIdx.y);
+    if (bx < nb1)
+        colsum_partial_block<T, VEC>(X1, R, C1, rows_per_chunk, partial1, bx, by);
     else
-        colsum_partial_block<T, VEC>(X2, R, C2, rows_per_chunk, partial2, blockIdx.x - nb1, blockIdx.y);
+        colsum_partial_block<T, VEC>(X2, R, C2, rows_per_chunk, partial2, bx - nb1, by);
 }
 
 // Column sums, pass 2: out[c] = Σ over chunks of partial[chunk][c]. Block
