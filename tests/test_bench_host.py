@@ -32,3 +32,15 @@ def test_fallback_has_no_sustained_figure():
 def test_default_workload_is_the_largest():
     args = bench.parse_args([])
     assert args.config == "175b"
+
+
+def test_schedule_summary_in_the_bench_line():
+    """config.schedules names each product's planned schedule (host-side
+    plan; 148 SMs without a GPU): the 175B-class row products on the
+    stream-K tail, the four bf16 row products dynamic, the weight
+    gradients static; the 7B-class step static whole tiles throughout."""
+    s = bench.plan_summary(2048, 12288, 49152, 8, "bf16")
+    assert s == {"F1": "whole tiles, dynamic", "F2": "stream-K tail, dynamic",
+                 "B2": "whole tiles, dynamic", "B3": "whole tiles", "B4": "whole tiles",
+                 "B5": "stream-K tail, dynamic"}
+    assert set(bench.plan_summary(8192, 4096, 16384, 2, "bf16").values()) == {"whole tiles"}
